@@ -1,0 +1,209 @@
+"""Python binding of the B200 mask-aware attention library (libfm_b200.so).
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels behind the C ABI declared in ``include/fm.h``.  PyTorch supplies device
+memory (the caller's tensors and the workspaces allocated here) and the
+current CUDA stream.  There is no CPU fallback: if the library is missing or
+cannot be loaded, ``lib()`` raises.
+
+Entry points (same names as the C ABI):
+  fm_build_mask_meta(lts, lte, uts, ute, n_q)      -> MaskMeta
+  fm_localize(vecs, chunk_start, chunk_len)         -> 4 tensors [R, B, Hm, N]
+  fm_attn_fwd(q, k, v, meta, vecs, scale)           -> (o, lse)
+  fm_attn_bwd(q, k, v, o, lse, do, meta, vecs, scale) -> (dq, dk, dv)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfm_b200.so")
+_lib = None
+
+FM_OK, FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA, FM_ERR_DEVICE_TIMEOUT = range(6)
+TILE = 128
+
+
+class FmError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} (status {code})")
+
+
+class MaskDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hm", ctypes.c_int32), ("n_q", ctypes.c_int32), ("n_k", ctypes.c_int32),
+                ("tile_q", ctypes.c_int32), ("tile_k", ctypes.c_int32)]
+
+
+class MaskMetaC(ctypes.Structure):
+    _fields_ = [("d", MaskDesc), ("tile_minmax", ctypes.c_void_p), ("row_count", ctypes.c_void_p),
+                ("row_entries", ctypes.c_void_p), ("col_count", ctypes.c_void_p),
+                ("col_entries", ctypes.c_void_p), ("tile_class", ctypes.c_void_p)]
+
+
+class AttnArgs(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("n_q", ctypes.c_int32), ("n_k", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p)]
+
+
+VecArray = ctypes.c_void_p * 4
+
+
+def lib():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with mask_aware_flash_b200._build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        L.fm_mask_meta_workspace_bytes.argtypes = [ctypes.POINTER(MaskDesc)]
+        L.fm_mask_meta_workspace_bytes.restype = sz
+        L.fm_build_mask_meta.argtypes = [ctypes.POINTER(MaskDesc), vp, vp, vp, vp, vp, sz, ctypes.POINTER(MaskMetaC),
+                                         vp]
+        L.fm_build_mask_meta.restype = ctypes.c_int
+        L.fm_localize.argtypes = [i32, i32, i32, VecArray, i32, i32, ctypes.POINTER(ctypes.c_int32),
+                                  ctypes.POINTER(ctypes.c_int32), VecArray, vp]
+        L.fm_localize.restype = ctypes.c_int
+        L.fm_attn_fwd.argtypes = [ctypes.POINTER(AttnArgs), ctypes.POINTER(MaskMetaC), VecArray, vp, vp, vp]
+        L.fm_attn_fwd.restype = ctypes.c_int
+        L.fm_attn_bwd_workspace_bytes.argtypes = [ctypes.POINTER(AttnArgs)]
+        L.fm_attn_bwd_workspace_bytes.restype = sz
+        L.fm_attn_bwd.argtypes = [ctypes.POINTER(AttnArgs), ctypes.POINTER(MaskMetaC), VecArray, vp, vp, vp, vp, vp,
+                                  vp, vp, sz, vp]
+        L.fm_attn_bwd.restype = ctypes.c_int
+        L.fm_get_device_status.argtypes = [vp]
+        L.fm_get_device_status.restype = ctypes.c_int
+        L.fm_status_string.argtypes = [ctypes.c_int]
+        L.fm_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().fm_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != FM_OK:
+        raise FmError(code, what)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _vecs(vecs):
+    return VecArray(*[None if v is None else v.data_ptr() for v in vecs])
+
+
+class MaskMeta:
+    """Tile metadata (views into an owned workspace tensor)."""
+
+    def __init__(self, desc: MaskDesc, ws: torch.Tensor, c: MaskMetaC):
+        self.desc, self.ws, self.c = desc, ws, c
+        B, Hm, n_q, n_k = desc.B, desc.Hm, desc.n_q, desc.n_k
+        self.T_q, self.T_k = -(-n_q // TILE), -(-n_k // TILE)
+        base = ws.data_ptr()
+
+        def view(ptr, dtype, shape):
+            n = 1
+            for s in shape:
+                n *= s
+            off = ptr - base
+            itemsize = torch.empty(0, dtype=dtype).element_size()
+            return ws[off:off + n * itemsize].view(dtype).view(*shape)
+
+        self.tile_minmax = view(c.tile_minmax, torch.int32, (B, Hm, self.T_k, 8))
+        self.row_count = view(c.row_count, torch.int32, (B, Hm, self.T_q))
+        self.row_entries = view(c.row_entries, torch.int32, (B, Hm, self.T_q, self.T_k))
+        self.col_count = view(c.col_count, torch.int32, (B, Hm, self.T_k))
+        self.col_entries = view(c.col_entries, torch.int32, (B, Hm, self.T_k, self.T_q))
+        self.tile_class = view(c.tile_class, torch.uint8, (B, Hm, self.T_q, self.T_k))
+
+
+def fm_mask_meta_workspace_bytes(B, Hm, n_q, n_k) -> int:
+    d = MaskDesc(B, Hm, n_q, n_k, TILE, TILE)
+    return int(lib().fm_mask_meta_workspace_bytes(ctypes.byref(d)))
+
+
+def fm_build_mask_meta(lts, lte, uts, ute, n_q: int, stream=None) -> MaskMeta:
+    """Vectors: int32 CUDA tensors [B, Hm, n_k] (or None = canonical empty)."""
+    ref = next(v for v in (lts, lte, uts, ute) if v is not None)
+    B, Hm, n_k = ref.shape
+    d = MaskDesc(B, Hm, n_q, n_k, TILE, TILE)
+    nbytes = lib().fm_mask_meta_workspace_bytes(ctypes.byref(d))
+    if nbytes == 0:
+        raise FmError(FM_ERR_INVALID_ARG, "fm_mask_meta_workspace_bytes")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=ref.device)
+    c = MaskMetaC()
+    _check(lib().fm_build_mask_meta(ctypes.byref(d), _ptr(lts), _ptr(lte), _ptr(uts), _ptr(ute), _ptr(ws), nbytes,
+                                    ctypes.byref(c), _stream(stream)), "fm_build_mask_meta")
+    return MaskMeta(d, ws, c)
+
+
+def fm_localize(vecs, chunk_start, chunk_len, stream=None):
+    """vecs: 4 int32 CUDA tensors [B, Hm, N]; chunk_start / chunk_len: [R, C] host ints.
+    Returns 4 int32 tensors [R, B, Hm, N]."""
+    import numpy as np
+    cs = np.ascontiguousarray(np.asarray(chunk_start, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(chunk_len, dtype=np.int32))
+    R, C = cs.shape
+    B, Hm, N = vecs[0].shape
+    outs = [torch.empty((R, B, Hm, N), dtype=torch.int32, device=vecs[0].device) for _ in range(4)]
+    _check(lib().fm_localize(B, Hm, N, _vecs(vecs), R, C, cs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                             cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _vecs(outs), _stream(stream)),
+           "fm_localize")
+    return outs
+
+
+def _args(q, k, v, scale) -> AttnArgs:
+    B, n_q, H, D = q.shape
+    return AttnArgs(B, H, n_q, k.shape[1], D, 0, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr())
+
+
+def fm_attn_fwd(q, k, v, meta: MaskMeta, vecs, scale, o=None, lse=None, stream=None):
+    """q [B, n_q, H, D], k/v [B, n_k, H, D] bf16 CUDA tensors -> o (bf16), lse [B, H, n_q] fp32."""
+    B, n_q, H, D = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
+    a = _args(q, k, v, scale)
+    _check(lib().fm_attn_fwd(ctypes.byref(a), ctypes.byref(meta.c), _vecs(vecs), _ptr(o), _ptr(lse),
+                             _stream(stream)), "fm_attn_fwd")
+    return o, lse
+
+
+def fm_attn_bwd_workspace_bytes(q, k, v, scale=1.0) -> int:
+    a = _args(q, k, v, scale)
+    return int(lib().fm_attn_bwd_workspace_bytes(ctypes.byref(a)))
+
+
+def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=None, dv=None, ws=None,
+                stream=None):
+    """Gradients (bf16) of the masked attention; ws: optional uint8 CUDA workspace."""
+    a = _args(q, k, v, scale)
+    nbytes = lib().fm_attn_bwd_workspace_bytes(ctypes.byref(a))
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(lib().fm_attn_bwd(ctypes.byref(a), ctypes.byref(meta.c), _vecs(vecs), _ptr(o), _ptr(lse), _ptr(do),
+                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)), "fm_attn_bwd")
+    return dq, dk, dv
+
+
+def fm_get_device_status(stream=None) -> int:
+    return int(lib().fm_get_device_status(_stream(stream)))

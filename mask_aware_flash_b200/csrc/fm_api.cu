@@ -1,0 +1,93 @@
+// Host-side plumbing shared by the entry points: status strings, the
+// per-device status word, and TMA tensor-map encoding.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "fm_common.cuh"
+
+namespace fm {
+
+// Latched device-side error (FM_ERR_DEVICE_TIMEOUT << 16 | site), one per device.
+__device__ int g_fm_status;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn get_encode() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+}  // namespace
+
+int* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fm_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+// 4-D map over a [B, n, H, D] bf16 tensor: dims (D, H, n, B), box (64, 1, box_rows, 1),
+// 128-byte swizzle (one 64-element row of the box = one swizzle span).
+bool encode_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t n, uint64_t B,
+                         uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {D, H, n, B};
+  cuuint64_t strides[3] = {D * 2, H * D * 2, n * H * D * 2};
+  cuuint32_t box[4] = {64, 1, box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace fm
+
+extern "C" {
+
+const char* fm_status_string(fm_status s) {
+  switch (s) {
+    case FM_OK: return "ok";
+    case FM_ERR_INVALID_ARG: return "invalid argument";
+    case FM_ERR_UNSUPPORTED: return "unsupported problem shape or type";
+    case FM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FM_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case FM_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out on the device";
+  }
+  return "unknown status";
+}
+
+fm_status fm_get_device_status(fm_stream_t stream) {
+  int* p = fm::device_status_ptr();
+  if (!p) return FM_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FM_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FM_ERR_CUDA;
+  if (v != 0 && cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FM_ERR_CUDA;
+  return v == 0 ? FM_OK : static_cast<fm_status>(v >> 16);
+}
+
+}  // extern "C"

@@ -1,0 +1,501 @@
+// Mask-aware attention backward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// The pages report the backward only as a measured speed-up (zicq.com summary,
+// end-to-end training paragraph: "attention forward and backward computation
+// speed increased by 24.5%-44.9%"); they give no design.  This kernel applies
+// the same tile classes as the forward (explainer, tile paragraph): each key
+// tile walks its column list of non-skip query tiles and applies the
+// row-interval test only on partial tiles.
+//
+// Per key tile of 128 keys (one CTA), per 64-row query sub-tile:
+//   S^T  = K Q^T        (tcgen05, M=128 keys, N=64 queries)      -> TMEM
+//   dP^T = V dO^T       (tcgen05)                                -> TMEM
+//   P^T  = 2^(S^T scale log2e - LSE2), masked entries 0         (warps 0-3)
+//   dS^T = P^T (dP^T - D_i)                                     (warps 0-3)
+//   dV  += P^T dO       (P^T read from TMEM)                    -> TMEM
+//   dK  += dS^T Q       (dS^T from shared memory)               -> TMEM
+//   dQ^T = K^T dS^T     (per sub-tile)                          -> TMEM -> fp32
+//        vector reductions into a global accumulator            (warps 4-7)
+// Warp 8 issues TMA loads, warp 9 issues the MMAs.  A preprocess kernel forms
+// D_i = dO_i.O_i and the log2-domain LSE and clears the accumulator; a final
+// kernel scales the accumulator into dQ (bf16).
+#include "fm_common.cuh"
+
+namespace fm {
+fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4]);
+
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kBQ = 64;  // query rows per backward sub-tile
+constexpr int kBwdThreads = 320;
+constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kPosInf = __builtin_huge_valf();
+
+struct BwdParams {
+  const int32_t* col_count;    // [B, Hm, T_k]
+  const int32_t* col_entries;  // [B, Hm, T_k, T_q]
+  const int32_t* vec[4];       // [B, Hm, n_k] or null
+  const float* lse2;           // [B, H, n_q] log2-domain LSE, +inf on empty rows
+  const float* dvec;           // [B, H, n_q] D_i = dO_i . O_i
+  float* dq_acc;               // [B, H, n_q/64][16][D][4] fp32
+  __nv_bfloat16* dk;           // [B, n_k, H, D]
+  __nv_bfloat16* dv;
+  int* status;
+  int B, H, Hm, n_q, n_k, T_q, T_k;
+  float scale, scale_log2;
+};
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kK = 0;                       // 128 x 128 bf16 (D=64: upper half kept zero, see dQ^T)
+  static constexpr int kV = kK + kTile * 128 * 2;
+  static constexpr int kQ = kV + kTile * D * 2;      // 2 stages x 64 x D
+  static constexpr int kQStage = kBQ * D * 2;
+  static constexpr int kDO = kQ + 2 * kQStage;       // 2 stages x 64 x D
+  static constexpr int kDS = kDO + 2 * kQStage;      // dS^T: 128 keys x 64 queries bf16
+  static constexpr int kStats = kDS + kTile * kBQ * 2;  // 2 stages x (64 lse2 + 64 D_i) fp32
+  static constexpr int kBar = kStats + 2 * 2 * kBQ * 4;
+  enum { KV_FULL, QDO_FULL0, QDO_FULL1, QDO_EMPTY0, QDO_EMPTY1, SDP_FULL, DS_READY, DS_EMPTY, DQ_FULL, DQ_EMPTY,
+         ACC_FULL, DRAIN, kNumBars };
+  static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort, [2] zero flag
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const BwdParams p) {
+  using S = BwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = (int)blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
+  const int64_t bh = (int64_t)b * p.H + h;
+  const int cnt = __ldg(p.col_count + bhm * p.T_k + kt);
+  const int nsub = 2 * cnt;  // two 64-row sub-tiles per listed 128-row query tile
+  const int32_t* entries = p.col_entries + (bhm * p.T_k + kt) * p.T_q;
+
+  const uint32_t bar0 = smem_u32(smem + S::kBar);
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + S::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  const volatile int* never = reinterpret_cast<const volatile int*>(misc + 2);
+  const uint32_t k_s = smem_u32(smem + S::kK), v_s = smem_u32(smem + S::kV);
+  const uint32_t q_s = smem_u32(smem + S::kQ), do_s = smem_u32(smem + S::kDO), ds_s = smem_u32(smem + S::kDS);
+  const float* stats = reinterpret_cast<const float*>(smem + S::kStats);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(S::KV_FULL), 1);
+    mbar_init(bar(S::QDO_FULL0), 1);
+    mbar_init(bar(S::QDO_FULL1), 1);
+    mbar_init(bar(S::QDO_EMPTY0), 1);
+    mbar_init(bar(S::QDO_EMPTY1), 1);
+    mbar_init(bar(S::SDP_FULL), 1);
+    mbar_init(bar(S::DS_READY), kTile);
+    mbar_init(bar(S::DS_EMPTY), 1);
+    mbar_init(bar(S::DQ_FULL), 1);
+    mbar_init(bar(S::DQ_EMPTY), kTile);
+    mbar_init(bar(S::ACC_FULL), 1);
+    mbar_init(bar(S::DRAIN), 1);
+    *abort_flag = 0;
+    misc[2] = 0;
+    fence_barrier_init();
+  }
+  if (D == 64) {  // K^T as a 128-row MMA operand: rows d >= 64 read this zero block
+    uint4* z = reinterpret_cast<uint4*>(smem + S::kK + kTile * 64 * 2);
+    for (int t = threadIdx.x; t < kTile * 64 * 2 / 16; t += blockDim.x) z[t] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const uint32_t tS = tmem, tdP = tmem + 64, tdQ = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ load role
+    if (lane == 0 && cnt > 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(bar(S::KV_FULL), 2 * kTile * D * 2);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_4d(k_s + c * 16384, &tm_k, bar(S::KV_FULL), c * 64, h, kt * kTile, b);
+        tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * 64, h, kt * kTile, b);
+      }
+      for (int i = 0; i < nsub; ++i) {
+        const int st = i & 1;
+        if (i >= 2 && !mbar_wait(bar(S::QDO_EMPTY0 + st), ((i >> 1) - 1) & 1, abort_flag)) {
+          record_failure(p.status, abort_flag, 11);
+          break;
+        }
+        const int ent = ld_nc_i32(entries + (i >> 1));
+        const int q0 = (ent >> 1) * kTile + (i & 1) * kBQ;
+        const uint32_t fb = bar(S::QDO_FULL0 + st);
+        mbar_arrive_expect_tx(fb, 2 * S::kQStage + 2 * kBQ * 4);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(q_s + st * S::kQStage + c * 8192, &tm_q, fb, c * 64, h, q0, b);
+          tma_load_4d(do_s + st * S::kQStage + c * 8192, &tm_do, fb, c * 64, h, q0, b);
+        }
+        bulk_load(smem_u32(stats + st * 2 * kBQ), p.lse2 + bh * p.n_q + q0, kBQ * 4, fb);
+        bulk_load(smem_u32(stats + st * 2 * kBQ + kBQ), p.dvec + bh * p.n_q + q0, kBQ * 4, fb);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------- MMA role
+    if (lane == 0 && cnt > 0) {
+      constexpr uint32_t kIdSdp = idesc_bf16(128, kBQ, false, false);  // S^T, dP^T: [key][q]
+      constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);     // dV, dK: [key][d], B MN-major
+      constexpr uint32_t kIdDq = idesc_bf16(128, kBQ, true, true);     // dQ^T: [d][q], A and B MN-major
+      bool ok = mbar_wait(bar(S::KV_FULL), 0, abort_flag);
+      for (int i = 0; ok && i < nsub; ++i) {
+        const int st = i & 1;
+        const uint32_t qs = q_s + st * S::kQStage, dos = do_s + st * S::kQStage;
+        if (!mbar_wait(bar(S::QDO_FULL0 + st), (i >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t okv = (k >> 2) * 16384 + (k & 3) * 32, oq = (k >> 2) * 8192 + (k & 3) * 32;
+          umma_ss(tS, smem_desc(k_s + okv, 16, 1024), smem_desc(qs + oq, 16, 1024), kIdSdp, k > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t okv = (k >> 2) * 16384 + (k & 3) * 32, oq = (k >> 2) * 8192 + (k & 3) * 32;
+          umma_ss(tdP, smem_desc(v_s + okv, 16, 1024), smem_desc(dos + oq, 16, 1024), kIdSdp, k > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(S::SDP_FULL));
+        if (!mbar_wait(bar(S::DS_READY), i & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dV += P^T dO (P^T bf16 in TMEM, 16 queries = 8 columns per step; dO MN-major)
+#pragma unroll
+        for (int k = 0; k < kBQ / 16; ++k)
+          umma_ts(tdV, tS + k * 8, smem_desc(dos + k * 2048, 8192, 1024), kIdAcc, (i > 0 || k > 0) ? 1u : 0u);
+        // dK += dS^T Q (dS^T K-major in smem, one swizzle atom wide; Q MN-major)
+#pragma unroll
+        for (int k = 0; k < kBQ / 16; ++k)
+          umma_ss(tdK, smem_desc(ds_s + k * 32, 16, 1024), smem_desc(qs + k * 2048, 8192, 1024), kIdAcc,
+                  (i > 0 || k > 0) ? 1u : 0u);
+        if (i > 0 && !mbar_wait(bar(S::DQ_EMPTY), (i - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dQ^T = K^T dS^T (K^T: M = d, MN-major; dS^T as B: N = q, MN-major; 16 keys per step)
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k)
+          umma_ss(tdQ, smem_desc(k_s + k * 2048, 16384, 1024), smem_desc(ds_s + k * 2048, 16384, 1024), kIdDq,
+                  k > 0 ? 1u : 0u);
+        umma_commit(bar(S::DQ_FULL));
+        umma_commit(bar(S::QDO_EMPTY0 + st));
+        umma_commit(bar(S::DS_EMPTY));
+      }
+      if (!ok) record_failure(p.status, abort_flag, 12);
+      umma_commit(bar(S::ACC_FULL));
+      umma_commit(bar(S::DRAIN));
+      mbar_wait(bar(S::DRAIN), 0, never);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------ P^T / dS^T role (row = key)
+    const int r = threadIdx.x;
+    const int64_t j = (int64_t)kt * kTile + r;
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const int64_t voff = bhm * p.n_k + j;
+    const int32_t lts = p.vec[0] ? __ldg(p.vec[0] + voff) : p.n_q, lte = p.vec[1] ? __ldg(p.vec[1] + voff) : p.n_q;
+    const int32_t uts = p.vec[2] ? __ldg(p.vec[2] + voff) : 0, ute = p.vec[3] ? __ldg(p.vec[3] + voff) : 0;
+    uint8_t* ds_row = smem + S::kDS + r * 128;
+    bool ok = true;
+    for (int i = 0; i < nsub; ++i) {
+      const int st = i & 1;
+      const int ent = ld_nc_i32(entries + (i >> 1));
+      const int q0 = (ent >> 1) * kTile + (i & 1) * kBQ;
+      const bool partial = ent & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(S::SDP_FULL), i & 1, abort_flag));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(S::QDO_FULL0 + st), (i >> 1) & 1, abort_flag));
+      if (!ok) break;
+      // dS^T buffer free: the previous sub-tile's dK / dQ^T MMAs have read it
+      // (their commit precedes this sub-tile's S^T/dP^T commit, so this wait is free)
+      if (i > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DS_EMPTY), (i - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      const float* l2 = stats + st * 2 * kBQ;
+      const float* dd = l2 + kBQ;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sr[32], dr[32], pk[16], dk[16];
+        tmem_ld32(tS + lane_addr + cc * 32, sr);
+        tmem_ld32(tdP + lane_addr + cc * 32, dr);
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qc = cc * 32 + c + u;
+            const int64_t q = q0 + qc;
+            float pr = ex2(__uint_as_float(sr[c + u]) * p.scale_log2 - l2[qc]);
+            if (partial && ((lts <= q && q < lte) || (uts <= q && q < ute))) pr = 0.f;
+            pv[u] = pr;
+            dsv[u] = pr * (__uint_as_float(dr[c + u]) - dd[qc]);
+          }
+          pk[c >> 1] = pack_bf16(pv[0], pv[1]);
+          dk[c >> 1] = pack_bf16(dsv[0], dsv[1]);
+        }
+        // P^T (bf16 pairs) over S^T columns [16 cc, 16 cc + 16): S^T columns >= 32 cc + 32 are still unread
+        tmem_st16(tS + lane_addr + cc * 16, pk);
+        // dS^T row r, queries [32 cc, 32 cc + 32): four 16-byte chunks, 128-byte swizzle (chunk c at c ^ (r & 7))
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = cc * 4 + c;
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(S::DS_READY));
+    }
+    if (!ok) record_failure(p.status, abort_flag, 13);
+  } else {
+    // ------------------------------------- dQ drain role (row = d), warps 4-7
+    const int d = threadIdx.x - 128;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q * D;
+    bool ok = true;
+    for (int i = 0; i < nsub; ++i) {
+      const int ent = ld_nc_i32(entries + (i >> 1));
+      const int q0 = (ent >> 1) * kTile + (i & 1) * kBQ;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DQ_FULL), i & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t a0[32], a1[32];
+      tmem_ld32(tdQ + lane_addr, a0);
+      tmem_ld32(tdQ + lane_addr + 32, a1);
+      tc_fence_before();
+      mbar_arrive(bar(S::DQ_EMPTY));
+      if (d < D) {
+        float* blk = acc_bh + (int64_t)q0 * D;  // [16 groups of 4 queries][D][4]
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          red_add_v4(blk + (g * D + d) * 4, __uint_as_float(a0[4 * g]), __uint_as_float(a0[4 * g + 1]),
+                     __uint_as_float(a0[4 * g + 2]), __uint_as_float(a0[4 * g + 3]));
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          red_add_v4(blk + ((g + 8) * D + d) * 4, __uint_as_float(a1[4 * g]), __uint_as_float(a1[4 * g + 1]),
+                     __uint_as_float(a1[4 * g + 2]), __uint_as_float(a1[4 * g + 3]));
+      }
+    }
+    if (!ok) record_failure(p.status, abort_flag, 14);
+  }
+
+  // ---------------------------------------------- epilogue: dV (warps 0-3), dK (warps 4-7)
+  if (warp < 8) {
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    const bool is_dk = warp >= 4;
+    bool have = false;
+    if (cnt > 0) {
+      have = __all_sync(0xffffffffu, mbar_wait(bar(S::ACC_FULL), 0, abort_flag));
+      tc_fence_after();
+    }
+    const float mul = is_dk ? p.scale : 1.f;
+    __nv_bfloat16* out = (is_dk ? p.dk : p.dv) + (((int64_t)b * p.n_k + (int64_t)kt * kTile + r) * p.H + h) * D;
+    const uint32_t tsrc = (is_dk ? tdK : tdV) + lane_addr;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t a[32];
+      if (have) {
+        tmem_ld32(tsrc + cc * 32, a);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) a[c] = 0u;
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2)
+        pk[c >> 1] = pack_bf16(__uint_as_float(a[c]) * mul, __uint_as_float(a[c + 1]) * mul);
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4)
+        st_global_v4(out + cc * 32 + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D_i = dO_i . O_i, log2-domain LSE (+inf for empty rows so that P = 0), and
+// a cleared dQ accumulator.  One thread per (b, i, h) row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout,
+                                                       const float* __restrict__ lse, float* __restrict__ lse2,
+                                                       float* __restrict__ dvec, float* __restrict__ acc, int B,
+                                                       int H, int n_q) {
+  const int64_t rows = (int64_t)B * n_q * H;
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < rows) {
+    const int h = (int)(t % H);
+    const int64_t bi = t / H;
+    const int i = (int)(bi % n_q), b = (int)(bi / n_q);
+    const uint4* po = reinterpret_cast<const uint4*>(o + t * D);
+    const uint4* pd = reinterpret_cast<const uint4*>(dout + t * D);
+    float s = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 a = __ldg(po + c), g = __ldg(pd + c);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[u]));
+        const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[u]));
+        s = fmaf(fa.x, fg.x, s);
+        s = fmaf(fa.y, fg.y, s);
+      }
+    }
+    const int64_t out = ((int64_t)b * H + h) * n_q + i;
+    dvec[out] = s;
+    const float l = lse[out];
+    lse2[out] = (l == kNegInf) ? kPosInf : l * 1.4426950408889634f;
+  }
+  // clear the accumulator (B*H*n_q*D floats), grid-stride in float4
+  float4* a4 = reinterpret_cast<float4*>(acc);
+  const int64_t n4 = rows * D / 4;
+  for (int64_t k = t; k < n4; k += (int64_t)gridDim.x * blockDim.x) a4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dQ[b, i, h, :] = scale * acc (accumulator layout [B,H,n_q/64][16][D][4]); 8 d per thread.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                                                     int B, int H, int n_q, float scale) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t total = (int64_t)B * n_q * H * (D / 8);
+  if (t >= total) return;
+  const int d0 = (int)(t % (D / 8)) * 8;
+  const int64_t row = t / (D / 8);  // (b, i, h) in output order
+  const int h = (int)(row % H);
+  const int64_t bi = row / H;
+  const int i = (int)(bi % n_q), b = (int)(bi / n_q);
+  const float* blk = acc + (((int64_t)b * H + h) * n_q + (i & ~63)) * D;
+  const int g = (i & 63) >> 2, u = i & 3;
+  uint32_t w[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float x0 = __ldg(blk + (g * D + d0 + 2 * c) * 4 + u) * scale;
+    const float x1 = __ldg(blk + (g * D + d0 + 2 * c + 1) * 4 + u) * scale;
+    w[c] = pack_bf16(x0, x1);
+  }
+  st_global_v4(dq + row * D + d0, w[0], w[1], w[2], w[3]);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdLayout {
+  size_t acc, lse2, dvec, total;
+};
+
+BwdLayout bwd_layout(const fm_attn_args* a) {
+  BwdLayout L;
+  const size_t rows = (size_t)a->B * a->H * a->n_q;
+  L.acc = 0;
+  L.lse2 = align256(rows * a->D * 4);
+  L.dvec = L.lse2 + align256(rows * 4);
+  L.total = L.dvec + align256(rows * 4);
+  return L;
+}
+
+template <int D>
+fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws, cudaStream_t stream) {
+  using S = BwdSmem<D>;
+  const BwdLayout L = bwd_layout(a);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* acc = reinterpret_cast<float*>(w + L.acc);
+  float* lse2 = reinterpret_cast<float*>(w + L.lse2);
+  float* dvec = reinterpret_cast<float*>(w + L.dvec);
+  CUtensorMap tq, tdo, tk, tv;
+  if (!encode_tmap_bf16_4d(&tq, a->q, D, a->H, a->n_q, a->B, kBQ) ||
+      !encode_tmap_bf16_4d(&tdo, dout, D, a->H, a->n_q, a->B, kBQ) ||
+      !encode_tmap_bf16_4d(&tk, a->k, D, a->H, a->n_k, a->B, kTile) ||
+      !encode_tmap_bf16_4d(&tv, a->v, D, a->H, a->n_k, a->B, kTile))
+    return FM_ERR_CUDA;
+  const int64_t rows = (int64_t)a->B * a->n_q * a->H;
+  bwd_prep_kernel<D><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec, acc, a->B,
+      a->H, a->n_q);
+  BwdParams p;
+  p.col_count = meta->col_count;
+  p.col_entries = meta->col_entries;
+  for (int c = 0; c < 4; ++c) p.vec[c] = vec ? vec[c] : nullptr;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.dq_acc = acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = device_status_ptr();
+  p.B = a->B;
+  p.H = a->H;
+  p.Hm = meta->d.Hm;
+  p.n_q = a->n_q;
+  p.n_k = a->n_k;
+  p.T_q = a->n_q / kTile;
+  p.T_k = a->n_k / kTile;
+  p.scale = a->scale;
+  p.scale_log2 = a->scale * 1.4426950408889634f;
+  if (cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) != cudaSuccess)
+    return FM_ERR_CUDA;
+  bwd_kernel<D><<<dim3(p.T_k, p.H, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, p);
+  const int64_t cvt = rows * (D / 8);
+  bwd_dq_kernel<D><<<(unsigned)((cvt + 255) / 256), 256, 0, stream>>>(acc, static_cast<__nv_bfloat16*>(dq), a->B,
+                                                                       a->H, a->n_q, a->scale);
+  return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fm
+
+extern "C" {
+
+size_t fm_attn_bwd_workspace_bytes(const fm_attn_args* a) {
+  if (!a || a->B < 1 || a->H < 1 || a->n_q < 1 || (a->D != 64 && a->D != 128)) return 0;
+  return fm::bwd_layout(a).total;
+}
+
+fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], const void* o,
+                      const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                      fm_stream_t stream) {
+  fm_status st = fm::check_attn_args(a, meta, vec);
+  if (st != FM_OK) return st;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(dout) |
+                       reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
+                       reinterpret_cast<uintptr_t>(dv);
+  if (!o || !lse || !dout || !dq || !dk || !dv || (al & 15) || (reinterpret_cast<uintptr_t>(lse) & 3))
+    return FM_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) || ws_bytes < fm_attn_bwd_workspace_bytes(a))
+    return FM_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return a->D == 64 ? fm::launch_bwd<64>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s)
+                    : fm::launch_bwd<128>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA path (through the C ABI) against the oracle on the same
+seeded inputs.  Bit-exact for tile metadata and localized vectors; for the
+attention: O max-abs <= 1e-2, LSE abs <= 1e-3 on live rows (exactly -inf and
+O exactly 0 on fully masked rows), dQ/dK/dV max-abs error relative to the
+oracle's max-abs <= 2e-2 per (b, h)."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, G_TOL = 1e-2, 1e-3, 2e-2
+
+
+@pytest.fixture(scope="module")
+def fm():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mask_aware_flash_b200 import _build
+    _build.build()
+    import mask_aware_flash_b200 as m
+    m.lib()
+    return m
+
+
+def _bf16_tensor(bits):
+    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    return t.cuda()
+
+
+def _inputs(B, n_q, n_k, H, D, seed):
+    qb = synth.normal_bf16_bits(seed, 1, (B, n_q, H, D))
+    kb = synth.normal_bf16_bits(seed, 2, (B, n_k, H, D))
+    vb = synth.normal_bf16_bits(seed, 3, (B, n_k, H, D))
+    db = synth.normal_bf16_bits(seed, 4, (B, n_q, H, D))
+    host = [synth.bf16_bits_to_f32(x) for x in (qb, kb, vb, db)]
+    dev = [_bf16_tensor(x) for x in (qb, kb, vb, db)]
+    return host, dev
+
+
+def _vec_tensors(vecs, B, Hm, n_k):
+    """1-D (or [B, Hm, n_k]) int32 vectors -> CUDA tensors [B, Hm, n_k]; None stays None."""
+    return [None if v is None else
+            torch.from_numpy(np.ascontiguousarray(np.broadcast_to(np.asarray(v, np.int32), (B, Hm, n_k)))).cuda()
+            for v in vecs]
+
+
+def _host_vecs(vt):
+    return [None if v is None else v.cpu().numpy() for v in vt]
+
+
+# ---------------------------------------------------------------------------- metadata
+def _check_meta(fm, vt, n_q, n_k):
+    meta = fm.fm_build_mask_meta(*vt, n_q=n_q)
+    torch.cuda.synchronize()
+    hv = _host_vecs(vt)
+    B, Hm = meta.desc.B, meta.desc.Hm
+    for b in range(B):
+        for hm in range(Hm):
+            ref = oracle.tile_meta(n_q, n_k, *[None if v is None else v[b, hm] for v in hv])
+            np.testing.assert_array_equal(meta.tile_minmax[b, hm].cpu().numpy(), ref["minmax"])
+            np.testing.assert_array_equal(meta.tile_class[b, hm].cpu().numpy(), ref["cls"])
+            rc = meta.row_count[b, hm].cpu().numpy()
+            np.testing.assert_array_equal(rc, ref["row_count"])
+            re_ = meta.row_entries[b, hm].cpu().numpy()
+            for qt in range(len(rc)):
+                np.testing.assert_array_equal(re_[qt, :rc[qt]], ref["row_entries"][qt, :rc[qt]])
+            cc = meta.col_count[b, hm].cpu().numpy()
+            np.testing.assert_array_equal(cc, ref["col_count"])
+            ce = meta.col_entries[b, hm].cpu().numpy()
+            for kt in range(len(cc)):
+                np.testing.assert_array_equal(ce[kt, :cc[kt]], ref["col_entries"][kt, :cc[kt]])
+    return meta
+
+
+@pytest.mark.parametrize("family", synth.SWEEP_FAMILIES)
+def test_meta_bitexact_families(fm, family):
+    n = 2048
+    spec = synth.make_family(family, n, 77)
+    vt = _vec_tensors(spec.vectors(), 2, 1, n)
+    _check_meta(fm, vt, n, n)
+
+
+def test_meta_bitexact_random_ragged(fm):
+    r = np.random.default_rng(5)
+    for (n_q, n_k, B, Hm) in [(300, 517, 2, 3), (128, 1000, 1, 1), (1001, 129, 3, 2), (5000, 4500, 1, 2)]:
+        vecs = [r.integers(-50, n_q + 50, (B, Hm, n_k)).astype(np.int32) for _ in range(4)]
+        vt = [torch.from_numpy(v).cuda() for v in vecs]
+        _check_meta(fm, vt, n_q, n_k)
+
+
+def test_meta_null_vectors(fm):
+    n = 512
+    spec = synth.mask_causal(n)
+    vt = [None, None, None] + _vec_tensors([spec.ute], 1, 1, n)
+    meta = _check_meta(fm, vt, n, n)
+    assert int(meta.tile_class.eq(1).sum()) == 4
+
+
+def test_meta_causal_128k_closed_form(fm):
+    n = 131072
+    T = n // 128
+    spec = synth.mask_causal(n)
+    meta = fm.fm_build_mask_meta(*_vec_tensors(spec.vectors(), 1, 1, n), n_q=n)
+    cls = meta.tile_class[0, 0]
+    assert int(cls.eq(0).sum()) == T * (T - 1) // 2
+    assert int(cls.eq(1).sum()) == T
+    assert int(cls.eq(2).sum()) == T * (T - 1) // 2
+    assert int(meta.row_count.sum()) == T * (T + 1) // 2
+
+
+# ---------------------------------------------------------------------------- localization
+def test_localize_bitexact(fm):
+    N, nch = 4096, 16
+    chunk = N // nch
+    R = nch // 2
+    starts = [[r * chunk, (nch - 1 - r) * chunk] for r in range(R)]
+    lens = [[chunk, chunk]] * R
+    r = np.random.default_rng(9)
+    vecs = [r.integers(-100, N + 100, (2, 1, N)).astype(np.int32) for _ in range(4)]
+    spec = synth.make_family("causal_document", N, 3)
+    vecs[0][1, 0] = spec.lts  # one batch row with a real mask
+    vecs[3][1, 0] = spec.ute
+    out = fm.fm_localize([torch.from_numpy(v).cuda() for v in vecs], starts, lens)
+    torch.cuda.synchronize()
+    for c in range(4):
+        got = out[c].cpu().numpy()
+        for rr in range(R):
+            for b in range(2):
+                exp = oracle.localize(vecs[c][b, 0], starts[rr], lens[rr])
+                np.testing.assert_array_equal(got[rr, b, 0], exp)
+
+
+# ---------------------------------------------------------------------------- attention
+def _run_attention(fm, B, H, n_q, n_k, D, vecs_np, Hm, seed, scale=None, bwd=True):
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    host, dev = _inputs(B, n_q, n_k, H, D, seed)
+    vt = [None if v is None else torch.from_numpy(np.ascontiguousarray(v, np.int32)).cuda() for v in vecs_np]
+    meta = fm.fm_build_mask_meta(*vt, n_q=n_q)
+    o, lse = fm.fm_attn_fwd(dev[0], dev[1], dev[2], meta, vt, scale)
+    res = {"o": o, "lse": lse, "host": host, "meta": meta, "vt": vt, "scale": scale}
+    if bwd:
+        dq, dk, dv = fm.fm_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], meta, vt, scale)
+        res.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert fm.fm_get_device_status() == 0
+    return res
+
+
+def _compare(res, vecs_np, Hm, heads=None, rows=None, cols=None, bwd=True):
+    q, k, v, do = res["host"]
+    B, n_q, H, D = q.shape
+    o = res["o"].float().cpu().numpy()
+    lse = res["lse"].cpu().numpy()
+    if bwd:
+        dq, dk, dv = (res[x].float().cpu().numpy() for x in ("dq", "dk", "dv"))
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for (b, h) in heads:
+        ref = oracle.attention_head(q, k, v, vecs_np, b, h, res["scale"], rows=rows,
+                                    cols=(np.arange(k.shape[1]) if (cols is None and bwd) else cols),
+                                    dout=do if bwd else None, Hm=Hm)
+        rr = ref["rows"]
+        live = np.isfinite(ref["lse"])
+        err_o = np.abs(o[b, rr, h] - ref["o"]).max()
+        assert err_o <= O_TOL, f"O max-abs {err_o} at (b={b}, h={h})"
+        if live.any():
+            err_l = np.abs(lse[b, h, rr][live] - ref["lse"][live]).max()
+            assert err_l <= LSE_TOL, f"LSE {err_l}"
+        assert np.all(np.isneginf(lse[b, h, rr][~live])), "dead rows need LSE = -inf"
+        assert np.all(o[b, rr, h][~live] == 0.0), "dead rows need O = 0"
+        if bwd:
+            for name, got, exp in (("dq", dq[b, rr, h], ref["dq"]), ("dk", dk[b, ref["cols"], h], ref["dk"]),
+                                   ("dv", dv[b, ref["cols"], h], ref["dv"])):
+                scale = max(np.abs(exp).max(), 1e-30)
+                err = np.abs(got - exp).max() / scale
+                assert err <= G_TOL, f"{name} rel-to-max error {err} at (b={b}, h={h})"
+
+
+def _vec_stack(spec, B, Hm):
+    return [np.ascontiguousarray(np.broadcast_to(x, (B, Hm, x.shape[-1]))) for x in spec.vectors()]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_tiny_causal_document(fm, D):
+    """B=1, H=2, n=256, 3 seeded documents, causal inside each."""
+    n = 256
+    docs = synth.cut_segments(synth.Rng(1000), n, 3)
+    spec = synth.mask_causal_document(n, docs)
+    vecs = _vec_stack(spec, 1, 1)
+    res = _run_attention(fm, 1, 2, n, n, D, vecs, 1, seed=1000)
+    _compare(res, vecs, 1)
+
+
+@pytest.mark.parametrize("family", ["full", "causal", "sliding_window_2k", "share_question", "random_eviction",
+                                    "global_sliding", "prefix_lm_document", "causal_blockwise"])
+def test_families_n640(fm, family):
+    n = 640  # five tiles: full, partial and skipped tiles
+    spec = synth.make_family(family, n, 31)
+    vecs = _vec_stack(spec, 1, 1)
+    res = _run_attention(fm, 1, 2, n, n, 128, vecs, 1, seed=2)
+    _compare(res, vecs, 1)
+
+
+def test_dead_rows_and_cross_lengths(fm):
+    n_q, n_k = 256, 512
+    r = np.random.default_rng(3)
+    lts = r.integers(0, n_q, n_k).astype(np.int32)
+    lte = r.integers(0, n_q + 1, n_k).astype(np.int32)
+    uts = np.zeros(n_k, np.int32)
+    ute = r.integers(0, n_q, n_k).astype(np.int32)
+    lts[:] = np.minimum(lts, 100)   # rows 100..139 are masked by every key
+    lte[:] = np.maximum(lte, 140)
+    vecs = [x[None, None] for x in (lts, lte, uts, ute)]
+    res = _run_attention(fm, 1, 2, n_q, n_k, 128, vecs, 1, seed=4)
+    _compare(res, vecs, 1)
+    assert np.all(res["dq"].float().cpu().numpy()[0, 100:140] == 0.0)
+
+
+def test_per_head_vectors_and_null(fm):
+    n, H = 384, 2
+    a, b_ = synth.mask_causal(n), synth.make_family("bidir_document", n, 5)
+    vecs = [np.stack([x, y])[None] for x, y in zip(a.vectors(), b_.vectors())]  # [1, 2, n]
+    res = _run_attention(fm, 1, H, n, n, 128, vecs, 2, seed=6)
+    _compare(res, vecs, 2)
+    vecs_null = [None, None, None, synth.mask_causal(n).ute[None, None]]
+    res = _run_attention(fm, 1, H, n, n, 128, vecs_null, 1, seed=7)
+    _compare(res, vecs_null, 1)
+
+
+def test_forward_deterministic(fm):
+    n = 1024
+    spec = synth.make_family("causal_document", n, 8)
+    vecs = _vec_stack(spec, 1, 1)
+    r1 = _run_attention(fm, 1, 4, n, n, 128, vecs, 1, seed=9, bwd=False)
+    r2 = _run_attention(fm, 1, 4, n, n, 128, vecs, 1, seed=9, bwd=False)
+    assert torch.equal(r1["o"], r2["o"]) and torch.equal(r1["lse"], r2["lse"])
+
+
+def _sample(n, count, seed, extra=()):
+    rng = synth.Rng(seed)
+    idx = set(rng.sample_distinct(0, n - 1, min(count, n)))
+    idx.update(extra)
+    return np.array(sorted(idx), dtype=np.int32)
+
+
+@pytest.mark.parametrize("mask", ["sliding_window", "causal_document"])
+def test_n8192_sampled(fm, mask):
+    """B=2, H=16, n=8192, D=128: (a) causal sliding window w=1024, (b) causal
+    documents with lengths ~ U[512, 4096]; checked on seeded samples of 512 rows
+    and 512 columns for two heads."""
+    n, B, H, D = 8192, 2, 16, 128
+    if mask == "sliding_window":
+        spec = synth.mask_sliding_window(n, 1024)
+    else:
+        spec = synth.mask_causal_document(n, synth.draw_docs(synth.Rng(2001), n, 512, 4096))
+    vecs = _vec_stack(spec, B, 1)
+    res = _run_attention(fm, B, H, n, n, D, vecs, 1, seed=2000 + (mask == "causal_document"))
+    rows = _sample(n, 512, 11, extra=(0, n - 1))
+    cols = _sample(n, 512, 12, extra=(0, n - 1))
+    _compare(res, vecs, 1, heads=[(0, 0), (1, 15)], rows=rows, cols=cols)
+
+
+def test_localized_forward_equals_global_rows(fm):
+    """Clip-shift-max + rank-local forward: each simulated rank's output rows are
+    bitwise equal to the corresponding rows of the global forward."""
+    N, nch, H, D = 4096, 8, 2, 128
+    chunk = N // nch
+    spec = synth.mask_causal_document(N, synth.draw_docs(synth.Rng(5), N, 256, 1024))
+    host, dev = _inputs(1, N, N, H, D, 50)
+    vt = [torch.from_numpy(np.ascontiguousarray(x[None, None])).cuda() for x in spec.vectors()]
+    scale = 1.0 / math.sqrt(D)
+    gmeta = fm.fm_build_mask_meta(*vt, n_q=N)
+    go, glse = fm.fm_attn_fwd(dev[0], dev[1], dev[2], gmeta, vt, scale)
+    R = nch // 2
+    starts = [[r * chunk, (nch - 1 - r) * chunk] for r in range(R)]
+    lens = [[chunk, chunk]] * R
+    loc = fm.fm_localize(vt, starts, lens)
+    for r in range(R):
+        rows = torch.cat([torch.arange(s, s + chunk) for s in starts[r]]).cuda()
+        ql = dev[0][:, rows].contiguous()
+        lv = [x[r].contiguous() for x in loc]
+        lmeta = fm.fm_build_mask_meta(*lv, n_q=2 * chunk)
+        lo, llse = fm.fm_attn_fwd(ql, dev[1], dev[2], lmeta, lv, scale)
+        torch.cuda.synchronize()
+        assert torch.equal(lo, go[:, rows]), f"rank {r}: O differs"
+        assert torch.equal(llse, glse[:, :, rows]), f"rank {r}: LSE differs"
+    assert fm.fm_get_device_status() == 0

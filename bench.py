@@ -1,0 +1,419 @@
+"""Benchmark of the mask-aware attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+for each mask of the workload, the tile metadata pass, the forward and the
+backward; plus one clip-shift-max localization of the batch's vectors to 8
+simulated context-parallel ranks (dual-chunk assignment).
+
+Default workload (N=1): n = 8192, B = 2, H = 16, D = 128, bf16, Q/K/V/dO ~ N(0,1),
+masks (a) causal sliding window w = 1024 and (b) causal documents with lengths
+~ U[512, 4096] (seeded per batch row).
+
+Metric: effective TFLOP/s counting only unmasked score entries
+(forward 4*D*U, backward 10*D*U per (b, h), U = unmasked (i, j) pairs).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--config n8192|n32768|n131072]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "mask-aware attn effective TFLOPs fwd/bwd (unmasked FLOPs), % of BF16 peak"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="n8192", choices=["n8192", "n32768", "n131072"])
+    ap.add_argument("--masks", default=None, help="comma list of mask names (default: the config's)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- workload
+def workload(config: str, rank: int, masks_arg=None):
+    if config == "n8192":
+        n, B, H, D = 8192, 2, 16, 128
+        masks = ["sliding_window_1024", "causal_document_512_4096"]
+        desc = "n=8192 B=2 H=16 D=128 bf16; masks: causal sliding window w=1024, causal documents L~U[512,4096]"
+    elif config == "n32768":
+        n, B, H, D = 32768, 1, 32, 128
+        masks = ["prefix_lm", "share_question"]
+        desc = "n=32768 B=1 H=32 D=128 bf16; masks: prefix-LM, share-question"
+    else:
+        n, B, H, D = 131072, 1, 16, 128
+        masks = ["causal", "sliding_window_2k"]
+        desc = "n=131072 B=1 H=16 D=128 bf16; masks: causal, causal sliding window 2K"
+    if masks_arg:
+        masks = masks_arg.split(",")
+        desc = desc.split(";")[0] + "; masks: " + ", ".join(masks)
+    cfg_id = {"n8192": 2, "n32768": 3, "n131072": 4}[config]
+    specs = []
+    for m_idx, name in enumerate(masks):
+        rows = []
+        for b in range(B):
+            seed = 1000 * cfg_id + 10 * b + m_idx + 100000 * rank
+            if name == "sliding_window_1024":
+                s = synth.mask_sliding_window(n, 1024)
+            elif name == "causal_document_512_4096":
+                s = synth.mask_causal_document(n, synth.draw_docs(synth.Rng(seed), n, 512, 4096))
+            else:
+                s = synth.make_family(name, n, seed)
+            rows.append(s)
+        specs.append((name, rows))
+    return dict(n=n, B=B, H=H, D=D, masks=specs, desc=desc, seed=1000 * cfg_id + 100000 * rank)
+
+
+def unmasked_pairs(spec_rows, n):
+    """U per batch row from interval lengths (plain per-column count)."""
+    out = []
+    for s in spec_rows:
+        lts, lte, uts, ute = (x.astype(np.int64) for x in s.vectors())
+        a0, a1 = np.clip(lts, 0, n), np.clip(lte, 0, n)
+        b0, b1 = np.clip(uts, 0, n), np.clip(ute, 0, n)
+        la, lb = np.maximum(a1 - a0, 0), np.maximum(b1 - b0, 0)
+        ov = np.maximum(np.minimum(a1, b1) - np.maximum(a0, b0), 0) * ((la > 0) & (lb > 0))
+        out.append(int(np.sum(n - (la + lb - ov))))
+    return out
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index):
+        self.dev = dev_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for k, name in enumerate(names):
+                if f[5 + k].lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"]}
+        load = [x for x in sm if x > 0.5 * (mx or max(sm))] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p.get("bf16_tflops_sustained"), p["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def lib_hash():
+    h = hashlib.sha256()
+    for d in ("mask_aware_flash_b200/csrc",):
+        for f in sorted(os.listdir(os.path.join(ROOT, d))):
+            with open(os.path.join(ROOT, d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, config: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t[config][kernel]
+        return e["bytes_per_launch"] if e.get("source_hash") == lib_hash() else None
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+def cpu_baseline(wl, budget_s=15.0):
+    """The oracle as it stands, on the host cores: forward + dQ for sampled rows of
+    two heads per mask; effective TFLOP/s = 14 * D * (unmasked pairs of the sampled
+    rows) / time."""
+    import oracle
+    n, B, H, D = wl["n"], wl["B"], wl["H"], wl["D"]
+    scale = 1.0 / math.sqrt(D)
+    # inputs of the sampled heads only (the oracle reads q/k/v/do of (b, h))
+    q = synth.bf16_bits_to_f32(synth.normal_bf16_bits(wl["seed"], 1, (1, n, 1, D)))
+    k = synth.bf16_bits_to_f32(synth.normal_bf16_bits(wl["seed"], 2, (1, n, 1, D)))
+    v = synth.bf16_bits_to_f32(synth.normal_bf16_bits(wl["seed"], 3, (1, n, 1, D)))
+    do = synth.bf16_bits_to_f32(synth.normal_bf16_bits(wl["seed"], 4, (1, n, 1, D)))
+    rows_per_call = 128
+    done_pairs, t_used, calls = 0, 0.0, 0
+    rng = synth.Rng(wl["seed"] + 7)
+    while t_used < budget_s and calls < 100000:
+        name, specs = wl["masks"][calls % len(wl["masks"])]
+        s = specs[0]
+        rows = np.array(rng.sample_distinct(0, n - 1, rows_per_call), np.int32)
+        vecs = [x[None, None] for x in s.vectors()]
+        allowed_rows = 0
+        for i in rows:  # unmasked pairs of the sampled rows (interval test per key, vectorised)
+            lts, lte, uts, ute = s.vectors()
+            m = ((lts <= i) & (i < lte)) | ((uts <= i) & (i < ute))
+            allowed_rows += int(n - m.sum())
+        t0 = time.perf_counter()
+        oracle.attention_head(q, k, v, vecs, 0, 0, scale, rows=rows, dout=do)
+        t_used += time.perf_counter() - t0
+        done_pairs += allowed_rows
+        calls += 1
+    flops = 14.0 * D * done_pairs
+    return {"value": flops / t_used / 1e12, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{calls} oracle calls x {rows_per_call} sampled query rows (forward + dQ, fp64) of head (0,0) "
+                      f"of the workload's masks, {done_pairs} unmasked pairs in {t_used:.1f} s; "
+                      f"effective FLOPs = 14*D*pairs"}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import mask_aware_flash_b200 as fm
+    from mask_aware_flash_b200 import _build
+    _build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workload(args.config, rank, args.masks)
+    n, B, H, D = wl["n"], wl["B"], wl["H"], wl["D"]
+    scale = 1.0 / math.sqrt(D)
+
+    def bf16(t_id):
+        bits = synth.normal_bf16_bits(wl["seed"], t_id, (B, n, H, D))
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+    host = {name: bf16(t).pin_memory() for name, t in (("q", 1), ("k", 2), ("v", 3), ("do", 4))}
+    q, k, v, do = (host[x].to(dev) for x in ("q", "k", "v", "do"))
+    vec_host, vec_dev = [], []
+    for name, specs in wl["masks"]:
+        vs = [torch.from_numpy(np.stack([s.vectors()[c] for s in specs])[:, None, :].copy()).pin_memory()
+              for c in range(4)]
+        vec_host.append(vs)
+        vec_dev.append([x.to(dev) for x in vs])
+    # dual-chunk assignment of 16 chunks to 8 simulated ranks
+    nch = 16
+    chunk = n // nch
+    loc_starts = [[r * chunk, (nch - 1 - r) * chunk] for r in range(nch // 2)]
+    loc_lens = [[chunk, chunk]] * (nch // 2)
+    U = [unmasked_pairs(specs, n) for _, specs in wl["masks"]]
+    flops_fwd = sum(4.0 * D * u * H for us in U for u in us)
+    flops_bwd = sum(10.0 * D * u * H for us in U for u in us)
+
+    stream = torch.cuda.current_stream()
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, n), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bws = torch.empty(fm.fm_attn_bwd_workspace_bytes(q, k, v), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(rec=None):
+        launches = 0
+        loc_in = [vec_dev[0][c] for c in range(4)]
+        fm.fm_localize(loc_in, loc_starts, loc_lens)
+        launches += 1
+        for mi in range(len(wl["masks"])):
+            vt = vec_dev[mi]
+            if rec is not None:
+                rec["m0"][mi].record(stream)
+            meta = fm.fm_build_mask_meta(*vt, n_q=n)
+            if rec is not None:
+                rec["f0"][mi].record(stream)
+            fm.fm_attn_fwd(q, k, v, meta, vt, scale, o=o, lse=lse)
+            if rec is not None:
+                rec["f1"][mi].record(stream)
+            fm.fm_attn_bwd(q, k, v, o, lse, do, meta, vt, scale, dq=dq, dk=dk, dv=dv, ws=bws)
+            if rec is not None:
+                rec["b1"][mi].record(stream)
+            launches += 2 + 1 + 3
+        return launches
+
+    import torch.distributed as dist
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    nm = len(wl["masks"])
+    recs = [{key: [ev() for _ in range(nm)] for key in ("m0", "f0", "f1", "b1")} for _ in range(args.steps)]
+    starts, ends = [ev() for _ in range(args.steps)], [ev() for _ in range(args.steps)]
+    launches = 0
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize()
+        for s in range(args.steps):
+            flush.fill_(s & 0xFF)  # L2 flush between steps, outside the step events
+            starts[s].record(stream)
+            launches += step(recs[s])
+            ends[s].record(stream)
+        torch.cuda.synchronize()
+    step_ms = [starts[s].elapsed_time(ends[s]) for s in range(args.steps)]
+    fwd_ms = sum(recs[s]["f0"][m].elapsed_time(recs[s]["f1"][m]) for s in range(args.steps) for m in range(nm))
+    bwd_ms = sum(recs[s]["f1"][m].elapsed_time(recs[s]["b1"][m]) for s in range(args.steps) for m in range(nm))
+    meta_ms = sum(recs[s]["m0"][m].elapsed_time(recs[s]["f0"][m]) for s in range(args.steps) for m in range(nm))
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_ms, bwd_ms = t.tolist()
+    steps = args.steps
+    value = world * (flops_fwd + flops_bwd) * steps / (total_ms * 1e-3) / 1e12
+
+    # end-to-end through the public API with host buffers (H2D of inputs, D2H of results)
+    e2e = None
+    if not args.no_e2e:
+        out_host = {x: torch.empty_like(host["q"] if x in ("o", "dq") else host["k"]).pin_memory()
+                    for x in ("o", "dq", "dk", "dv")}
+        lse_host = torch.empty((B, H, n), dtype=torch.float32).pin_memory()
+        h2d = sum(host[x].numel() * 2 for x in host) + sum(t_.numel() * 4 for vs in vec_host for t_ in vs)
+        d2h = 4 * q.numel() * 2 + lse.numel() * 4
+
+        def e2e_step():
+            for x, dst in (("q", q), ("k", k), ("v", v), ("do", do)):
+                dst.copy_(host[x], non_blocking=True)
+            for mi, vs in enumerate(vec_host):
+                for c in range(4):
+                    vec_dev[mi][c].copy_(vs[c], non_blocking=True)
+            step()
+            for x, src in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+                out_host[x].copy_(src, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+
+        for _ in range(max(1, args.warmup // 2)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * (flops_fwd + flops_bwd) * steps / (te.item() * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    assert fm.fm_get_device_status() == 0, "device-side timeout during the bench"
+
+    burst, sustained, hbm, src = peaks()
+    fwd_tf = flops_fwd * steps / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = flops_bwd * steps / (bwd_ms * 1e-3) / 1e12
+    dominant = "bwd_kernel" if bwd_ms >= fwd_ms else "fwd_kernel"
+    ach = bwd_tf if dominant == "bwd_kernel" else fwd_tf
+    peak = burst
+    launches_per_traffic = {"fwd_kernel": B * H * (n // 128), "bwd_kernel": B * H * (n // 128)}
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), seeded masks)",
+        "config": {"workload": wl["desc"], "B": B, "H": H, "seq_len": n, "head_dim": D,
+                   "masks": [m for m, _ in wl["masks"]], "unmasked_pairs_per_head": U,
+                   "localize": "8 simulated ranks, dual-chunk, 16 chunks", "parallelism": f"replicas x{world}",
+                   "l2": "flushed between steps (256 MiB write outside the step events); inputs 256 MiB > L2"},
+        "fwd": {"effective_tflops": round(fwd_tf, 2), "frac_of_measured_burst": round(fwd_tf / burst, 4),
+                "frac_of_2250_nominal": round(fwd_tf / 2250.0, 4), "ms_per_step": round(fwd_ms / steps, 4)},
+        "bwd": {"effective_tflops": round(bwd_tf, 2), "frac_of_measured_burst": round(bwd_tf / burst, 4),
+                "frac_of_2250_nominal": round(bwd_tf / 2250.0, 4), "ms_per_step": round(bwd_ms / steps, 4),
+                "note": "includes the D_i preprocess and dQ convert kernels"},
+        "meta_ms_per_step": round(meta_ms / steps, 4),
+        "roofline": {"bound": "tensor", "kernel": dominant, "achieved": round(ach, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                     "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)",
+                     "traffic": traffic_for(dominant, args.config)},
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
+    }
+    return line, wl
+
+
+def run_reference(args):
+    wl = workload(args.config, 0, args.masks)
+    cb = cpu_baseline(wl, budget_s=max(5.0, min(20.0, 3.0 * args.steps)))
+    return {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), seeded masks)",
+            "config": {"workload": wl["desc"]}, "impl": "reference", "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    line, wl = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

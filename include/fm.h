@@ -174,6 +174,40 @@ fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int
                       void* ws, size_t ws_bytes, fm_stream_t stream);
 
 /*
+ * Size of the fixed device scratch used by fm_attn_bwd_noalloc: 32 MiB, held
+ * by every GPU that loads this library for as long as the process lives.
+ */
+#define FM_BWD_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * fm_attn_bwd without a caller-supplied workspace.  The paper has no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory when they call the backward: for example a plug-in inside an
+ * inference or training engine that plans every device buffer up front and
+ * exposes no workspace to its kernels, or a latency-critical loop that must not
+ * pay cudaMalloc's implicit device synchronisation.  It computes exactly what
+ * fm_attn_bwd computes, with the same arguments minus ws / ws_bytes; its
+ * scratch (fp32 dQ accumulator, per-row statistics) lives in one fixed device
+ * array of FM_BWD_NOALLOC_SCRATCH_BYTES bytes inside the library, and it calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *   - Limit: fm_attn_bwd_workspace_bytes(a) must not exceed
+ *     FM_BWD_NOALLOC_SCRATCH_BYTES (for D = 128 about 64K query rows in total,
+ *     B * H * n_q); larger problems are rejected with FM_ERR_WORKSPACE before
+ *     any launch.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array; it keeps the last call's
+ *     contents and each call clears what must start at zero.  Calls whose
+ *     kernels overlap on the GPU (different streams, no ordering between
+ *     them) race on the array and give wrong gradients: order them.
+ * Errors: as fm_attn_bwd, plus FM_ERR_CUDA if the address lookup fails.
+ */
+fm_status fm_attn_bwd_noalloc(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4],
+                              const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              fm_stream_t stream);
+
+/*
  * Reads and clears the current device's status word: FM_OK, or
  * FM_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since the last
  * call.  Synchronises `stream` (the one call that does).

@@ -19,6 +19,8 @@
 // Warp 8 issues TMA loads, warp 9 issues the MMAs.  A preprocess kernel forms
 // D_i = dO_i.O_i and the log2-domain LSE and clears the accumulator; a final
 // kernel scales the accumulator into dQ (bf16).
+#include <mutex>
+
 #include "fm_common.cuh"
 
 namespace fm {
@@ -499,3 +501,38 @@ fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free backward: the same kernels with their scratch in a fixed
+// device array owned by the library (see fm_attn_bwd_noalloc in fm.h).
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_bwd_noalloc_scratch[FM_BWD_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" fm_status fm_attn_bwd_noalloc(const fm_attn_args* a, const fm_mask_meta* meta,
+                                         const int32_t* const vec[4], const void* o, const float* lse,
+                                         const void* dout, void* dq, void* dk, void* dv, fm_stream_t stream) {
+  fm_status st = fm::check_attn_args(a, meta, vec);
+  if (st != FM_OK) return st;
+  if (fm_attn_bwd_workspace_bytes(a) > FM_BWD_NOALLOC_SCRATCH_BYTES) return FM_ERR_WORKSPACE;
+  void* ws = noalloc_scratch();
+  if (!ws) return FM_ERR_CUDA;
+  return fm_attn_bwd(a, meta, vec, o, lse, dout, dq, dk, dv, ws, FM_BWD_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -430,6 +430,7 @@ template <int D>
 fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], const void* o,
                      const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws, cudaStream_t stream) {
   using S = BwdSmem<D>;
+  static_assert(S::kAlloc <= 227 * 1024, "backward shared memory exceeds the per-CTA limit");
   const BwdLayout L = bwd_layout(a);
   uint8_t* w = static_cast<uint8_t*>(ws);
   float* acc = reinterpret_cast<float*>(w + L.acc);

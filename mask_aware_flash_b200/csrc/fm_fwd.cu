@@ -6,28 +6,36 @@
 // pages' Hopper kernel (paper abstract: three-role warp specialisation on the
 // FlashAttention-3 TMA/WGMMA pipeline) is prior art; this kernel is designed
 // for Blackwell:
-//   * one CTA per (query tile of 128 rows, head, batch), two CTAs per SM
-//     (256 TMEM columns and ~101 KB shared memory each), so the tensor core of
-//     an SM alternates between two independent softmax pipelines;
-//   * warp 4 (one lane) issues TMA loads of Q once and of K/V plus the tile's
-//     four boundary-vector slices (partial tiles only) for each entry of the
-//     query tile's block list;
-//   * warp 5 (one lane) issues tcgen05.mma: S = Q K^T into TMEM, then
-//     O += P V with P read straight from TMEM (bf16, aliased over S);
-//   * warps 0-3 (one thread per query row) read S from TMEM, apply the
-//     row-interval test on partial tiles, run the online softmax in the log2
-//     domain, write P back to TMEM, rescale O in TMEM when the row maximum
-//     grows, and finally normalise O and write O and LSE.
+//   * one CTA per (pair of 128-row query tiles, head, batch), one CTA per SM,
+//     512 TMEM columns: S0 | O0 | S1 | O1 (fp32, 128 lanes x 128 columns each);
+//   * the two query tiles walk the merged (union) block list of their two row
+//     lists and share every K/V tile, which TMA streams through a two-deep ring;
+//   * warp 8 (one lane) issues the TMA loads (Q once; per merged entry K, V and,
+//     when a partial tile needs it, the tile's slice of the four vectors);
+//   * warp 9 (one lane) issues tcgen05.mma in the order
+//       PV0(e), S0(e+1), PV1(e), S1(e+1)
+//     so the tensor core computes one tile's scores while the other tile's
+//     softmax runs (S = Q K^T into TMEM; O += P V with P, bf16, read from TMEM
+//     over the first half of the S columns);
+//   * warps 0-3 / 4-7 are the softmax of tile 0 / tile 1 (one thread per row):
+//     one TMEM read of the 128 scores, the row-interval test on partial tiles
+//     only, online softmax in the log2 domain with the running maximum moved
+//     only when it grows by more than 8 (O in TMEM is rescaled then), P written
+//     back to TMEM, and the epilogue O / l, LSE.
 // Every mbarrier wait is bounded; on a timeout the CTA records the failure in
 // the device status word and unwinds (no wait can hang the GPU).
+#include <climits>
+
 #include "fm_common.cuh"
 
 namespace fm {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kFwdThreads = 192;
+constexpr int kFwdThreads = 320;
+constexpr int kMaxList = 4096;  // key tiles per query tile held in shared memory (n_k <= 524288)
 constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 struct FwdParams {
   const int32_t* row_count;    // [B, Hm, T_q]
@@ -36,273 +44,361 @@ struct FwdParams {
   __nv_bfloat16* o;            // [B, n_q, H, D]
   float* lse;                  // [B, H, n_q]
   int* status;
-  int B, H, Hm, n_q, n_k, T_q, T_k;
-  float scale_log2;            // softmax scale * log2(e)
+  int B, H, Hm, n_q, n_k, T_q, T_k, n_pairs;
+  float scale_log2;            // softmax scale * log2(e), > 0
 };
 
 template <int D>
 struct FwdSmem {
   static constexpr int kTileBytes = kTile * D * 2;  // 128 rows x D bf16 (D/64 swizzle-atom columns)
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kTileBytes;
-  static constexpr int kMask = kV + kTileBytes;     // [2 buffers][4 vectors][128] int32
-  static constexpr int kBar = kMask + 2 * 4 * kTile * 4;
-  enum { Q_FULL, K_FULL, K_EMPTY, V_FULL, V_EMPTY, S_FULL, P_FULL, O_DONE, DRAIN, M_FULL0, M_FULL1, M_EMPTY0,
-         M_EMPTY1, kNumBars };
-  static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
+  static constexpr int kQ = 0;                      // Q0, Q1
+  static constexpr int kK = kQ + 2 * kTileBytes;    // K ring, 2 slots
+  static constexpr int kV = kK + 2 * kTileBytes;    // V ring, 2 slots
+  static constexpr int kMask = kV + 2 * kTileBytes; // [2 buffers][4 vectors][128] int32
+  static constexpr int kList = kMask + 2 * 4 * kTile * 4;  // two row lists, kMaxList uint16 each
+  static constexpr int kBar = kList + 2 * kMaxList * 2;
+  enum { Q_FULL, K_FULL0, K_FULL1, K_EMPTY0, K_EMPTY1, V_FULL0, V_FULL1, V_EMPTY0, V_EMPTY1, S_FULL0, S_FULL1,
+         P_FULL0, P_FULL1, O_DONE0, O_DONE1, M_FULL0, M_FULL1, M_EMPTY0, M_EMPTY1, DRAIN, kNumBars };
+  static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag, [2] zero
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;       // slack for 1024-byte alignment of the base
 };
 
+// Walks the union of two ascending row lists (entries (kt << 1) | partial).
+// Yields each key tile once with the class it has for each query tile
+// (0 skip, 1 partial, 2 full).  Every role runs its own copy over the same
+// shared-memory lists, so all roles see the same sequence.
+struct MergedList {
+  const uint16_t* a;
+  const uint16_t* b;
+  int na, nb, pa, pb;
+  __device__ __forceinline__ bool next(int& kt, int& c0, int& c1) {
+    const int ea = pa < na ? a[pa] : INT_MAX, eb = pb < nb ? b[pb] : INT_MAX;
+    const int ka = ea >> 1, kb = eb >> 1;
+    kt = min(ka, kb);
+    if (kt == (INT_MAX >> 1)) return false;
+    c0 = (ka == kt) ? ((ea & 1) ? 1 : 2) : 0;
+    c1 = (kb == kt) ? ((eb & 1) ? 1 : 2) : 0;
+    pa += (ka == kt);
+    pb += (kb == kt);
+    return true;
+  }
+};
+
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 2)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using S = FwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.T_q - 1 - (int)blockIdx.x;  // long (late causal) query tiles first
+  const int pair = p.n_pairs - 1 - (int)blockIdx.x;  // long (late causal) query tiles first
   const int h = blockIdx.y, b = blockIdx.z;
+  const int qt0 = 2 * pair, qt1 = 2 * pair + 1;
+  const bool has1 = qt1 < p.T_q;
   const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
-  const int cnt = __ldg(p.row_count + bhm * p.T_q + qt);
-  const int32_t* entries = p.row_entries + (bhm * p.T_q + qt) * p.T_k;
+  const int32_t* rows0 = p.row_entries + (bhm * p.T_q + qt0) * p.T_k;
+  const int32_t* rows1 = rows0 + p.T_k;
+  const int n0 = __ldg(p.row_count + bhm * p.T_q + qt0);
+  const int n1 = has1 ? __ldg(p.row_count + bhm * p.T_q + qt1) : 0;
 
   const uint32_t bar0 = smem_u32(smem + S::kBar);
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + S::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  const volatile int* never = reinterpret_cast<const volatile int*>(misc + 2);
   const uint32_t q_s = smem_u32(smem + S::kQ), k_s = smem_u32(smem + S::kK), v_s = smem_u32(smem + S::kV);
   const int32_t* mask_smem = reinterpret_cast<const int32_t*>(smem + S::kMask);
+  uint16_t* list0 = reinterpret_cast<uint16_t*>(smem + S::kList);
+  uint16_t* list1 = list0 + kMaxList;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(S::Q_FULL), 1);
-    mbar_init(bar(S::K_FULL), 1);
-    mbar_init(bar(S::K_EMPTY), 1);
-    mbar_init(bar(S::V_FULL), 1);
-    mbar_init(bar(S::V_EMPTY), 1);
-    mbar_init(bar(S::S_FULL), 1);
-    mbar_init(bar(S::P_FULL), kTile);
-    mbar_init(bar(S::O_DONE), 1);
-    mbar_init(bar(S::DRAIN), 1);
-    mbar_init(bar(S::M_FULL0), 1);
-    mbar_init(bar(S::M_FULL1), 1);
-    mbar_init(bar(S::M_EMPTY0), kTile);
-    mbar_init(bar(S::M_EMPTY1), kTile);
+    for (int k = 0; k < S::kNumBars; ++k) mbar_init(bar(k), 1);
+    mbar_init(bar(S::P_FULL0), kTile);
+    mbar_init(bar(S::P_FULL1), kTile);
+    mbar_init(bar(S::M_EMPTY0), 2 * kTile);
+    mbar_init(bar(S::M_EMPTY1), 2 * kTile);
     *abort_flag = 0;
     misc[2] = 0;  // a flag nothing raises: lets the final drain wait ignore aborts
     fence_barrier_init();
   }
-  if (warp == 5) {
-    tmem_alloc(smem_u32(misc), 256);
+  // both row lists into shared memory (coalesced)
+  for (int t = threadIdx.x; t < n0; t += kFwdThreads) list0[t] = (uint16_t)__ldg(rows0 + t);
+  for (int t = threadIdx.x; t < n1; t += kFwdThreads) list1[t] = (uint16_t)__ldg(rows1 + t);
+  if (warp == 9) {
+    tmem_alloc(smem_u32(misc), 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const bool any = (n0 + n1) > 0;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ load role
-    if (lane == 0 && cnt > 0) {
+    if (lane == 0 && any) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       int nvec = 0;
       for (int c = 0; c < 4; ++c) nvec += p.vec[c] ? 1 : 0;
-      mbar_arrive_expect_tx(bar(S::Q_FULL), S::kTileBytes);
-      for (int c = 0; c < D / 64; ++c) tma_load_4d(q_s + c * 16384, &tm_q, bar(S::Q_FULL), c * 64, h, qt * kTile, b);
-      int pm = 0;
-      for (int e = 0; e < cnt; ++e) {
-        const int ent = ld_nc_i32(entries + e);
-        const int kt = ent >> 1;
-        if (e > 0 && !mbar_wait(bar(S::K_EMPTY), (e - 1) & 1, abort_flag)) {
-          record_failure(p.status, abort_flag, 1);
+      mbar_arrive_expect_tx(bar(S::Q_FULL), (has1 ? 2 : 1) * S::kTileBytes);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_4d(q_s + c * 16384, &tm_q, bar(S::Q_FULL), c * 64, h, qt0 * kTile, b);
+        if (has1) tma_load_4d(q_s + S::kTileBytes + c * 16384, &tm_q, bar(S::Q_FULL), c * 64, h, qt1 * kTile, b);
+      }
+      MergedList it{list0, list1, n0, n1, 0, 0};
+      int kt, c0, c1, e = 0, mcount = 0;
+      bool ok = true;
+      while (it.next(kt, c0, c1)) {
+        const int slot = e & 1;
+        if (e >= 2 && !mbar_wait(bar(S::K_EMPTY0 + slot), ((e >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(S::K_FULL), S::kTileBytes);
-        for (int c = 0; c < D / 64; ++c) tma_load_4d(k_s + c * 16384, &tm_k, bar(S::K_FULL), c * 64, h, kt * kTile, b);
-        if (ent & 1) {
-          const int buf = pm & 1;
-          if (pm >= 2 && !mbar_wait(bar(S::M_EMPTY0 + buf), ((pm >> 1) - 1) & 1, abort_flag)) {
-            record_failure(p.status, abort_flag, 2);
+        mbar_arrive_expect_tx(bar(S::K_FULL0 + slot), S::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(k_s + slot * S::kTileBytes + c * 16384, &tm_k, bar(S::K_FULL0 + slot), c * 64, h, kt * kTile, b);
+        if (c0 == 1 || c1 == 1) {
+          const int mb = mcount & 1;
+          if (mcount >= 2 && !mbar_wait(bar(S::M_EMPTY0 + mb), ((mcount >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(S::M_FULL0 + buf), 512u * nvec);
+          mbar_arrive_expect_tx(bar(S::M_FULL0 + mb), 512u * nvec);
           for (int c = 0; c < 4; ++c)
             if (p.vec[c])
-              bulk_load(smem_u32(mask_smem + (buf * 4 + c) * kTile), p.vec[c] + bhm * p.n_k + (int64_t)kt * kTile,
-                        512u, bar(S::M_FULL0 + buf));
-          ++pm;
+              bulk_load(smem_u32(mask_smem + (mb * 4 + c) * kTile), p.vec[c] + bhm * p.n_k + (int64_t)kt * kTile,
+                        512u, bar(S::M_FULL0 + mb));
+          ++mcount;
         }
-        if (e > 0 && !mbar_wait(bar(S::V_EMPTY), (e - 1) & 1, abort_flag)) {
-          record_failure(p.status, abort_flag, 3);
+        if (e >= 2 && !mbar_wait(bar(S::V_EMPTY0 + slot), ((e >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(S::V_FULL), S::kTileBytes);
-        for (int c = 0; c < D / 64; ++c) tma_load_4d(v_s + c * 16384, &tm_v, bar(S::V_FULL), c * 64, h, kt * kTile, b);
+        mbar_arrive_expect_tx(bar(S::V_FULL0 + slot), S::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(v_s + slot * S::kTileBytes + c * 16384, &tm_v, bar(S::V_FULL0 + slot), c * 64, h, kt * kTile, b);
+        ++e;
       }
+      if (!ok) record_failure(p.status, abort_flag, 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA role
-    if (lane == 0 && cnt > 0) {
+    if (lane == 0 && any) {
       constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false, false);  // S[q][kv]: Q K-major, K K-major
       constexpr uint32_t kIdescPV = idesc_bf16(128, D, false, true);     // O[q][d]:  P (TMEM), V MN-major
+      MergedList it{list0, list1, n0, n1, 0, 0};
+      int kt, c0, c1, kn, n0c, n1c;
       bool ok = mbar_wait(bar(S::Q_FULL), 0, abort_flag);
-      for (int e = 0; ok && e < cnt; ++e) {
-        if (!mbar_wait(bar(S::K_FULL), e & 1, abort_flag)) {
+      bool has_cur = ok && it.next(kt, c0, c1);
+      int np[2] = {0, 0};  // P tiles consumed per query tile (p_full phases)
+      bool acc[2] = {false, false};
+      if (has_cur) {
+        ok = mbar_wait(bar(S::K_FULL0), 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t)
+            if (t ? c1 : c0) {
+              const uint32_t qa = q_s + t * S::kTileBytes, ka = k_s;
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k) {
+                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                umma_ss(tmem + t * 256, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), kIdescQK,
+                        k > 0 ? 1u : 0u);
+              }
+              umma_commit(bar(S::S_FULL0 + t));
+            }
+          umma_commit(bar(S::K_EMPTY0));
+        }
+      }
+      for (int e = 0; ok && has_cur; ++e) {
+        const bool has_next = it.next(kn, n0c, n1c);
+        const int slot = e & 1, nslot = (e + 1) & 1;
+        if (has_next && !mbar_wait(bar(S::K_FULL0 + nslot), ((e + 1) >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;  // swizzle-atom column, 16-element K step
-          umma_ss(tS, smem_desc(q_s + off, 16, 1024), smem_desc(k_s + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
-        }
-        umma_commit(bar(S::S_FULL));
-        umma_commit(bar(S::K_EMPTY));
-        if (!mbar_wait(bar(S::P_FULL), e & 1, abort_flag) || !mbar_wait(bar(S::V_FULL), e & 1, abort_flag)) {
+        if (!mbar_wait(bar(S::V_FULL0 + slot), (e >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
-        tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)  // 16 kv rows per step; P columns advance 8 (bf16 pairs)
-          umma_ts(tO, tS + k * 8, smem_desc(v_s + k * 2048, 16384, 1024), kIdescPV, (e > 0 || k > 0) ? 1u : 0u);
-        umma_commit(bar(S::O_DONE));
-        umma_commit(bar(S::V_EMPTY));
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t tS = tmem + t * 256, tO = tS + 128;
+          if (t ? c1 : c0) {  // O_t += P_t V(e)
+            if (!mbar_wait(bar(S::P_FULL0 + t), np[t] & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            ++np[t];
+            tc_fence_after();
+            const uint32_t va = v_s + slot * S::kTileBytes;
+#pragma unroll
+            for (int k = 0; k < kTile / 16; ++k)  // 16 kv rows per step; P columns advance 8 (bf16 pairs)
+              umma_ts(tO, tS + k * 8, smem_desc(va + k * 2048, 16384, 1024), kIdescPV, (acc[t] || k > 0) ? 1u : 0u);
+            umma_commit(bar(S::O_DONE0 + t));
+            acc[t] = true;
+          }
+          if (has_next && (t ? n1c : n0c)) {  // S_t = Q_t K(e+1)^T, after PV_t(e) has read P_t
+            const uint32_t qa = q_s + t * S::kTileBytes, ka = k_s + nslot * S::kTileBytes;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+              umma_ss(tS, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+            }
+            umma_commit(bar(S::S_FULL0 + t));
+          }
+        }
+        if (!ok) break;
+        umma_commit(bar(S::V_EMPTY0 + slot));
+        if (has_next) umma_commit(bar(S::K_EMPTY0 + nslot));
+        has_cur = has_next;
+        kt = kn;
+        c0 = n0c;
+        c1 = n1c;
       }
       if (!ok) record_failure(p.status, abort_flag, 4);
       // drain: every MMA issued above has finished before TMEM is released
       umma_commit(bar(S::DRAIN));
-      mbar_wait(bar(S::DRAIN), 0, reinterpret_cast<const volatile int*>(misc + 2));
+      mbar_wait(bar(S::DRAIN), 0, never);
     }
   } else {
     // ---------------------------------------------------------- softmax role
-    const int r = threadIdx.x;  // row in tile == TMEM lane
+    const int t = warp >> 2;                   // query tile of this warpgroup
+    const int r = threadIdx.x & 127;           // row in tile == TMEM lane
+    const int qt = t ? qt1 : qt0;
     const int64_t i = (int64_t)qt * kTile + r;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + t * 256 + lane_addr, tO = tS + 128;
     const bool has[4] = {p.vec[0] != nullptr, p.vec[1] != nullptr, p.vec[2] != nullptr, p.vec[3] != nullptr};
-    float m_run = kNegInf, l_run = 0.f;
-    int pm = 0;
+    float m_run = kNegInf, l_run = 0.f, lq_run = 0.f;
+    int j = 0, mcount = 0;
     bool ok = true;
-    for (int e = 0; e < cnt; ++e) {
-      const int ent = ld_nc_i32(entries + e);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(S::S_FULL), e & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      // row-interval test, partial tiles only
-      uint32_t mbits[4] = {0u, 0u, 0u, 0u};
-      if (ent & 1) {
-        const int buf = pm & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::M_FULL0 + buf), (pm >> 1) & 1, abort_flag));
-        if (!ok) break;
-        const int32_t* mv = mask_smem + buf * 4 * kTile;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t bits = 0u;
-#pragma unroll 8
-          for (int c = 0; c < 32; ++c) {
-            const int col = cc * 32 + c;
-            const int32_t lts = has[0] ? mv[col] : p.n_q, lte = has[1] ? mv[kTile + col] : p.n_q;
-            const int32_t uts = has[2] ? mv[2 * kTile + col] : 0, ute = has[3] ? mv[3 * kTile + col] : 0;
-            const bool msk = (lts <= i && i < lte) || (uts <= i && i < ute);
-            bits |= (msk ? 1u : 0u) << c;
-          }
-          mbits[cc] = bits;
-        }
-        mbar_arrive(bar(S::M_EMPTY0 + buf));
-        ++pm;
-      }
-      // pass 1: row maximum of the scaled scores (log2 domain)
-      float mx = kNegInf;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32];
-        tmem_ld32(tS + lane_addr + cc * 32, sr);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float t = ((mbits[cc] >> c) & 1u) ? kNegInf : __uint_as_float(sr[c]) * p.scale_log2;
-          mx = fmaxf(mx, t);
-        }
-      }
-      const float m_new = fmaxf(m_run, mx);
-      const float m_use = (m_new == kNegInf) ? 0.f : m_new;
-      const float alpha = ex2(m_run - m_use);
-      // pass 2: P = 2^(t - m) as bf16 pairs written over the first 64 S columns
-      float rs = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32];
-        tmem_ld32(tS + lane_addr + cc * 32, sr);
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float p0 = ((mbits[cc] >> c) & 1u) ? 0.f : ex2(__uint_as_float(sr[c]) * p.scale_log2 - m_use);
-          const float p1 = ((mbits[cc] >> (c + 1)) & 1u) ? 0.f : ex2(__uint_as_float(sr[c + 1]) * p.scale_log2 - m_use);
-          rs += p0 + p1;
-          pk[c >> 1] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tS + lane_addr + cc * 16, pk);
-      }
-      l_run = l_run * alpha + rs;
-      // rescale O when the running maximum moved (O holds sum over earlier tiles)
-      if (__any_sync(0xffffffffu, e > 0 && alpha != 1.f)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE), (e - 1) & 1, abort_flag));
+    MergedList it{list0, list1, n0, n1, 0, 0};
+    int kt, c0, c1;
+    const bool live_tile = (t == 0) || has1;
+    // A warpgroup without a query tile (odd tile count) still walks the list:
+    // both warpgroups release every shared mask buffer.
+    while (it.next(kt, c0, c1)) {
+      const int ct = t ? c1 : c0;
+      const bool has_mask = (c0 == 1 || c1 == 1);
+      const int mb = mcount & 1;
+      if (ct != 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::S_FULL0 + t), j & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
+        uint32_t s[128];
+        tmem_ld128(tS, s);
+        if (ct == 1) {
+          // row-interval test (partial tiles only): masked scores -> -inf
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(S::M_FULL0 + mb), (mcount >> 1) & 1, abort_flag));
+          if (!ok) break;
+          const int32_t* mv = mask_smem + mb * 4 * kTile;
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t orr[32];
-          tmem_ld32(tO + lane_addr + cc * 32, orr);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-          tmem_st32(tO + lane_addr + cc * 32, orr);
+          for (int c = 0; c < kTile; ++c) {
+            const int32_t lts = has[0] ? mv[c] : p.n_q, lte = has[1] ? mv[kTile + c] : p.n_q;
+            const int32_t uts = has[2] ? mv[2 * kTile + c] : 0, ute = has[3] ? mv[3 * kTile + c] : 0;
+            const bool msk = (lts <= i && i < lte) || (uts <= i && i < ute);
+            s[c] = msk ? __float_as_uint(kNegInf) : s[c];
+          }
         }
+        float mx0 = kNegInf, mx1 = kNegInf;
+#pragma unroll
+        for (int c = 0; c < kTile; c += 4) {
+          mx0 = fmax3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        }
+        const float m_tile = fmaxf(mx0, mx1) * p.scale_log2;
+        // move the running maximum only when it grows by more than the threshold
+        const bool move = (m_tile - m_run) > kRescaleThreshold;  // false when both are -inf
+        const float m_new = move ? m_tile : m_run;
+        const float alpha = move ? ex2(m_run - m_new) : 1.f;
+        const float m_use = (m_new == kNegInf) ? 0.f : m_new;
+        // rs: exact fp32 row sum (LSE); rq: sum of the bf16-rounded P the PV product
+        // actually uses (O is normalised by it, so O stays a convex combination of V rows)
+        float rs = 0.f, rq = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < kTile; c += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[c]), p.scale_log2, -m_use));
+          const float p1 = ex2(fmaf(__uint_as_float(s[c + 1]), p.scale_log2, -m_use));
+          rs += p0 + p1;
+          const uint32_t w = pack_bf16(p0, p1);
+          rq += bf16_lo(w) + bf16_hi(w);
+          pk[c >> 1] = w;
+        }
+        tmem_st64(tS, pk);
+        l_run = l_run * alpha + rs;
+        lq_run = lq_run * alpha + rq;
+        m_run = m_new;
+        if (__any_sync(0xffffffffu, move && j > 0)) {
+          // O holds the sum over earlier tiles: wait for the last PV, rescale in TMEM
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE0 + t), (j - 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t orr[32];
+            tmem_ld32(tO + cc * 32, orr);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+            tmem_st32(tO + cc * 32, orr);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(S::P_FULL0 + t));
+        ++j;
+      } else if (has_mask) {
+        // keep the two warpgroups in step on the shared mask buffers
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::M_FULL0 + mb), (mcount >> 1) & 1, abort_flag));
+        if (!ok) break;
       }
-      m_run = m_new;
-      tc_fence_before();
-      mbar_arrive(bar(S::P_FULL));
+      if (has_mask) {
+        mbar_arrive(bar(S::M_EMPTY0 + mb));
+        ++mcount;
+      }
     }
     if (!ok) record_failure(p.status, abort_flag, 5);
     // epilogue: O = O / l, LSE = (m + log2 l) ln 2; empty rows: O = 0, LSE = -inf
-    __nv_bfloat16* orow = p.o + (((int64_t)b * p.n_q + i) * p.H + h) * D;
-    const bool live = ok && cnt > 0 && l_run > 0.f;
-    bool have_o = false;
-    if (ok && cnt > 0) {
-      have_o = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE), (cnt - 1) & 1, abort_flag));
-      if (!have_o) record_failure(p.status, abort_flag, 6);
-      tc_fence_after();
-    }
-    const float inv = live ? 1.f / l_run : 0.f;
-#pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t orr[32];
-      if (have_o) {
-        tmem_ld32(tO + lane_addr + cc * 32, orr);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) orr[c] = 0u;
+    if (live_tile) {
+      __nv_bfloat16* orow = p.o + (((int64_t)b * p.n_q + i) * p.H + h) * D;
+      const bool live = ok && j > 0 && l_run > 0.f;
+      bool have_o = false;
+      if (ok && j > 0) {
+        have_o = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE0 + t), (j - 1) & 1, abort_flag));
+        if (!have_o) record_failure(p.status, abort_flag, 6);
+        tc_fence_after();
       }
-      uint32_t pk[16];
+      const float inv = live && lq_run > 0.f ? 1.f / lq_run : 0.f;
 #pragma unroll
-      for (int c = 0; c < 32; c += 2)
-        pk[c >> 1] = pack_bf16(__uint_as_float(orr[c]) * inv, __uint_as_float(orr[c + 1]) * inv);
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t orr[32];
+        if (have_o) {
+          tmem_ld32(tO + cc * 32, orr);
+        } else {
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4)
-        st_global_v4(orow + cc * 32 + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          for (int c = 0; c < 32; ++c) orr[c] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2)
+          pk[c >> 1] = pack_bf16(__uint_as_float(orr[c]) * inv, __uint_as_float(orr[c + 1]) * inv);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          st_global_v4(orow + cc * 32 + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+      p.lse[((int64_t)b * p.H + h) * p.n_q + i] = live ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
     }
-    p.lse[((int64_t)b * p.H + h) * p.n_q + i] = live ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -310,6 +406,7 @@ template <int D>
 fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], void* o,
                      float* lse, cudaStream_t stream) {
   using S = FwdSmem<D>;
+  static_assert(S::kAlloc <= 227 * 1024, "forward shared memory exceeds the per-CTA limit");
   CUtensorMap tq, tk, tv;
   if (!encode_tmap_bf16_4d(&tq, a->q, D, a->H, a->n_q, a->B, kTile) ||
       !encode_tmap_bf16_4d(&tk, a->k, D, a->H, a->n_k, a->B, kTile) ||
@@ -329,10 +426,11 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.n_k = a->n_k;
   p.T_q = a->n_q / kTile;
   p.T_k = a->n_k / kTile;
+  p.n_pairs = (p.T_q + 1) / 2;
   p.scale_log2 = a->scale * 1.4426950408889634f;
   if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) != cudaSuccess)
     return FM_ERR_CUDA;
-  fwd_kernel<D><<<dim3(p.T_q, p.H, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, p);
+  fwd_kernel<D><<<dim3(p.n_pairs, p.H, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 
@@ -342,10 +440,11 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
 fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4]) {
   if (!a || !meta) return FM_ERR_INVALID_ARG;
   if (a->B < 1 || a->H < 1 || a->n_q < 1 || a->n_k < 1 || a->B > 65535 || a->H > 65535) return FM_ERR_INVALID_ARG;
-  if (!(a->scale == a->scale)) return FM_ERR_INVALID_ARG;
+  if (!(a->scale > 0.f) || a->scale > 3.0e38f) return FM_ERR_INVALID_ARG;  // positive and finite
   if (a->dtype != 0) return FM_ERR_UNSUPPORTED;
   if (a->D != 64 && a->D != 128) return FM_ERR_UNSUPPORTED;
   if (a->n_q % kTile || a->n_k % kTile) return FM_ERR_UNSUPPORTED;
+  if (a->n_k / kTile > kMaxList) return FM_ERR_UNSUPPORTED;
   if (!a->q || !a->k || !a->v) return FM_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->k) | reinterpret_cast<uintptr_t>(a->v)) & 15)
     return FM_ERR_INVALID_ARG;

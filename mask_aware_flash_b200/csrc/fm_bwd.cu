@@ -31,6 +31,7 @@ namespace {
 constexpr int kTile = 128;
 constexpr int kBQ = 64;  // query rows per backward sub-tile
 constexpr int kBwdThreads = 320;
+constexpr int kMaxList = 4096;  // query tiles per key tile held in shared memory
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kPosInf = __builtin_huge_valf();
 
@@ -50,16 +51,19 @@ struct BwdParams {
 
 template <int D>
 struct BwdSmem {
+  static constexpr int kQStages = 3;
   static constexpr int kK = 0;                       // 128 x 128 bf16 (D=64: upper half kept zero, see dQ^T)
   static constexpr int kV = kK + kTile * 128 * 2;
-  static constexpr int kQ = kV + kTile * D * 2;      // 2 stages x 64 x D
-  static constexpr int kQStage = kBQ * D * 2;
-  static constexpr int kDO = kQ + 2 * kQStage;       // 2 stages x 64 x D
-  static constexpr int kDS = kDO + 2 * kQStage;      // dS^T: 128 keys x 64 queries bf16
-  static constexpr int kStats = kDS + kTile * kBQ * 2;  // 2 stages x (64 lse2 + 64 D_i) fp32
-  static constexpr int kBar = kStats + 2 * 2 * kBQ * 4;
-  enum { KV_FULL, QDO_FULL0, QDO_FULL1, QDO_EMPTY0, QDO_EMPTY1, SDP_FULL, DS_READY, DS_EMPTY, DQ_FULL, DQ_EMPTY,
-         ACC_FULL, DRAIN, kNumBars };
+  static constexpr int kQStage = kBQ * D * 2;        // one 64-row sub-tile of Q (or dO)
+  static constexpr int kQ = kV + kTile * D * 2;      // kQStages x Q
+  static constexpr int kDO = kQ + kQStages * kQStage;  // kQStages x dO
+  static constexpr int kDSBytes = kTile * kBQ * 2;   // dS^T: 128 keys x 64 queries bf16
+  static constexpr int kDS = kDO + kQStages * kQStage;  // 2 buffers
+  static constexpr int kStats = kDS + 2 * kDSBytes;  // kQStages x (64 lse2 + 64 D_i) fp32
+  static constexpr int kList = kStats + kQStages * 2 * kBQ * 4;  // column list, uint16
+  static constexpr int kBar = kList + kMaxList * 2;
+  enum { KV_FULL, QDO_FULL0, QDO_FULL1, QDO_FULL2, QDO_EMPTY0, QDO_EMPTY1, QDO_EMPTY2, SDP_FULL, DP_FREE,
+         DS_READY, DS_EMPTY0, DS_EMPTY1, DQ_FULL, DQ_EMPTY, ACC_FULL, DRAIN, kNumBars };
   static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort, [2] zero flag
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -71,6 +75,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const BwdParams p) {
   using S = BwdSmem<D>;
+  constexpr int NS = S::kQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,24 +95,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t k_s = smem_u32(smem + S::kK), v_s = smem_u32(smem + S::kV);
   const uint32_t q_s = smem_u32(smem + S::kQ), do_s = smem_u32(smem + S::kDO), ds_s = smem_u32(smem + S::kDS);
   const float* stats = reinterpret_cast<const float*>(smem + S::kStats);
+  uint16_t* list = reinterpret_cast<uint16_t*>(smem + S::kList);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(S::KV_FULL), 1);
-    mbar_init(bar(S::QDO_FULL0), 1);
-    mbar_init(bar(S::QDO_FULL1), 1);
-    mbar_init(bar(S::QDO_EMPTY0), 1);
-    mbar_init(bar(S::QDO_EMPTY1), 1);
-    mbar_init(bar(S::SDP_FULL), 1);
+    for (int k = 0; k < S::kNumBars; ++k) mbar_init(bar(k), 1);
+    mbar_init(bar(S::DP_FREE), kTile);
     mbar_init(bar(S::DS_READY), kTile);
-    mbar_init(bar(S::DS_EMPTY), 1);
-    mbar_init(bar(S::DQ_FULL), 1);
     mbar_init(bar(S::DQ_EMPTY), kTile);
-    mbar_init(bar(S::ACC_FULL), 1);
-    mbar_init(bar(S::DRAIN), 1);
     *abort_flag = 0;
     misc[2] = 0;
     fence_barrier_init();
   }
+  for (int t = threadIdx.x; t < cnt; t += kBwdThreads) list[t] = (uint16_t)__ldg(entries + t);
   if (D == 64) {  // K^T as a 128-row MMA operand: rows d >= 64 read this zero block
     uint4* z = reinterpret_cast<uint4*>(smem + S::kK + kTile * 64 * 2);
     for (int t = threadIdx.x; t < kTile * 64 * 2 / 16; t += blockDim.x) z[t] = make_uint4(0, 0, 0, 0);
@@ -121,7 +120,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  const uint32_t tS = tmem, tdP = tmem + 64, tdQ = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+  // TMEM columns: S^T / P^T double buffer [0,64) [64,128), dP^T [128,192), dQ^T [192,256), dV, dK
+  const uint32_t tdP = tmem + 128, tdQ = tmem + 192, tdV = tmem + 256, tdK = tmem + 384;
+  auto sub_q0 = [&](int i) { return (int)(list[i >> 1] >> 1) * kTile + (i & 1) * kBQ; };
 
   if (warp == 8) {
     // ------------------------------------------------------------ load role
@@ -136,13 +137,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * 64, h, kt * kTile, b);
       }
       for (int i = 0; i < nsub; ++i) {
-        const int st = i & 1;
-        if (i >= 2 && !mbar_wait(bar(S::QDO_EMPTY0 + st), ((i >> 1) - 1) & 1, abort_flag)) {
+        const int st = i % NS, use = i / NS;
+        if (use >= 1 && !mbar_wait(bar(S::QDO_EMPTY0 + st), (use - 1) & 1, abort_flag)) {
           record_failure(p.status, abort_flag, 11);
           break;
         }
-        const int ent = ld_nc_i32(entries + (i >> 1));
-        const int q0 = (ent >> 1) * kTile + (i & 1) * kBQ;
+        const int q0 = sub_q0(i);
         const uint32_t fb = bar(S::QDO_FULL0 + st);
         mbar_arrive_expect_tx(fb, 2 * S::kQStage + 2 * kBQ * 4);
         for (int c = 0; c < D / 64; ++c) {
@@ -159,40 +159,63 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t kIdSdp = idesc_bf16(128, kBQ, false, false);  // S^T, dP^T: [key][q]
       constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);     // dV, dK: [key][d], B MN-major
       constexpr uint32_t kIdDq = idesc_bf16(128, kBQ, true, true);     // dQ^T: [d][q], A and B MN-major
-      bool ok = mbar_wait(bar(S::KV_FULL), 0, abort_flag);
-      for (int i = 0; ok && i < nsub; ++i) {
-        const int st = i & 1;
-        const uint32_t qs = q_s + st * S::kQStage, dos = do_s + st * S::kQStage;
-        if (!mbar_wait(bar(S::QDO_FULL0 + st), (i >> 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      auto issue_s = [&](int i) {  // S^T_i = K Q_i^T
+        const uint32_t qs = q_s + (i % NS) * S::kQStage, tS = tmem + (i & 1) * 64;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t okv = (k >> 2) * 16384 + (k & 3) * 32, oq = (k >> 2) * 8192 + (k & 3) * 32;
           umma_ss(tS, smem_desc(k_s + okv, 16, 1024), smem_desc(qs + oq, 16, 1024), kIdSdp, k > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dp = [&](int i) {  // dP^T_i = V dO_i^T
+        const uint32_t dos = do_s + (i % NS) * S::kQStage;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t okv = (k >> 2) * 16384 + (k & 3) * 32, oq = (k >> 2) * 8192 + (k & 3) * 32;
           umma_ss(tdP, smem_desc(v_s + okv, 16, 1024), smem_desc(dos + oq, 16, 1024), kIdSdp, k > 0 ? 1u : 0u);
         }
+      };
+      bool ok = mbar_wait(bar(S::KV_FULL), 0, abort_flag) && mbar_wait(bar(S::QDO_FULL0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
         umma_commit(bar(S::SDP_FULL));
+      }
+      for (int i = 0; ok && i < nsub; ++i) {
+        const int st = i % NS, bi = i & 1;
+        if (i + 1 < nsub) {  // next sub-tile's S^T (other buffer) and dP^T, overlapping this sub-tile's softmax
+          if (!mbar_wait(bar(S::QDO_FULL0 + (i + 1) % NS), ((i + 1) / NS) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(i + 1);
+          if (!mbar_wait(bar(S::DP_FREE), i & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dp(i + 1);
+          umma_commit(bar(S::SDP_FULL));
+        }
         if (!mbar_wait(bar(S::DS_READY), i & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t qs = q_s + st * S::kQStage, dos = do_s + st * S::kQStage, dss = ds_s + bi * S::kDSBytes;
+        const uint32_t tP = tmem + bi * 64;
         // dV += P^T dO (P^T bf16 in TMEM, 16 queries = 8 columns per step; dO MN-major)
 #pragma unroll
         for (int k = 0; k < kBQ / 16; ++k)
-          umma_ts(tdV, tS + k * 8, smem_desc(dos + k * 2048, 8192, 1024), kIdAcc, (i > 0 || k > 0) ? 1u : 0u);
+          umma_ts(tdV, tP + k * 8, smem_desc(dos + k * 2048, 8192, 1024), kIdAcc, (i > 0 || k > 0) ? 1u : 0u);
         // dK += dS^T Q (dS^T K-major in smem, one swizzle atom wide; Q MN-major)
 #pragma unroll
         for (int k = 0; k < kBQ / 16; ++k)
-          umma_ss(tdK, smem_desc(ds_s + k * 32, 16, 1024), smem_desc(qs + k * 2048, 8192, 1024), kIdAcc,
+          umma_ss(tdK, smem_desc(dss + k * 32, 16, 1024), smem_desc(qs + k * 2048, 8192, 1024), kIdAcc,
                   (i > 0 || k > 0) ? 1u : 0u);
+        umma_commit(bar(S::QDO_EMPTY0 + st));
         if (i > 0 && !mbar_wait(bar(S::DQ_EMPTY), (i - 1) & 1, abort_flag)) {
           ok = false;
           break;
@@ -201,11 +224,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dQ^T = K^T dS^T (K^T: M = d, MN-major; dS^T as B: N = q, MN-major; 16 keys per step)
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          umma_ss(tdQ, smem_desc(k_s + k * 2048, 16384, 1024), smem_desc(ds_s + k * 2048, 16384, 1024), kIdDq,
+          umma_ss(tdQ, smem_desc(k_s + k * 2048, 16384, 1024), smem_desc(dss + k * 2048, 16384, 1024), kIdDq,
                   k > 0 ? 1u : 0u);
         umma_commit(bar(S::DQ_FULL));
-        umma_commit(bar(S::QDO_EMPTY0 + st));
-        umma_commit(bar(S::DS_EMPTY));
+        umma_commit(bar(S::DS_EMPTY0 + bi));
       }
       if (!ok) record_failure(p.status, abort_flag, 12);
       umma_commit(bar(S::ACC_FULL));
@@ -220,55 +242,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int64_t voff = bhm * p.n_k + j;
     const int32_t lts = p.vec[0] ? __ldg(p.vec[0] + voff) : p.n_q, lte = p.vec[1] ? __ldg(p.vec[1] + voff) : p.n_q;
     const int32_t uts = p.vec[2] ? __ldg(p.vec[2] + voff) : 0, ute = p.vec[3] ? __ldg(p.vec[3] + voff) : 0;
-    uint8_t* ds_row = smem + S::kDS + r * 128;
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
-      const int st = i & 1;
-      const int ent = ld_nc_i32(entries + (i >> 1));
-      const int q0 = (ent >> 1) * kTile + (i & 1) * kBQ;
-      const bool partial = ent & 1;
+      const int st = i % NS, bi = i & 1;
+      const int q0 = sub_q0(i);
+      const bool partial = list[i >> 1] & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(S::SDP_FULL), i & 1, abort_flag));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(S::QDO_FULL0 + st), (i >> 1) & 1, abort_flag));
       if (!ok) break;
-      // dS^T buffer free: the previous sub-tile's dK / dQ^T MMAs have read it
-      // (their commit precedes this sub-tile's S^T/dP^T commit, so this wait is free)
-      if (i > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DS_EMPTY), (i - 1) & 1, abort_flag));
+      tc_fence_after();
+      uint32_t sd[128];  // [0, 64): S^T row, [64, 128): dP^T row
+      tmem_ld64x2(tmem + bi * 64 + lane_addr, tdP + lane_addr, sd);
+      tc_fence_before();
+      mbar_arrive(bar(S::DP_FREE));  // dP^T columns may be overwritten by the next sub-tile
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(S::QDO_FULL0 + st), (i / NS) & 1, abort_flag));
+      if (!ok) break;
+      const float4* l2 = reinterpret_cast<const float4*>(stats + st * 2 * kBQ);
+      const float4* dd = l2 + kBQ / 4;
+      uint32_t pk[32], dk[32];
+#pragma unroll
+      for (int c4 = 0; c4 < kBQ / 4; ++c4) {
+        const float4 L = l2[c4], Dd = dd[c4];
+        const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dd.x, Dd.y, Dd.z, Dd.w};
+        float pv[4], dsv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int qc = c4 * 4 + u;
+          float pr = ex2(fmaf(__uint_as_float(sd[qc]), p.scale_log2, -lv[u]));  // 0 on empty rows (lse2 = +inf)
+          if (partial) {
+            const int64_t q = q0 + qc;
+            if ((lts <= q && q < lte) || (uts <= q && q < ute)) pr = 0.f;
+          }
+          pv[u] = pr;
+          dsv[u] = pr * (__uint_as_float(sd[64 + qc]) - dv[u]);
+        }
+        pk[2 * c4] = pack_bf16(pv[0], pv[1]);
+        pk[2 * c4 + 1] = pack_bf16(pv[2], pv[3]);
+        dk[2 * c4] = pack_bf16(dsv[0], dsv[1]);
+        dk[2 * c4 + 1] = pack_bf16(dsv[2], dsv[3]);
+      }
+      // P^T (bf16 pairs) over this buffer's first 32 S^T columns (all S^T values are in registers)
+      tmem_st32(tmem + bi * 64 + lane_addr, pk);
+      if (i >= 2) {  // dS^T buffer bi free: the dK / dQ^T MMAs of sub-tile i-2 have read it
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DS_EMPTY0 + bi), ((i >> 1) - 1) & 1, abort_flag));
         if (!ok) break;
       }
-      tc_fence_after();
-      const float* l2 = stats + st * 2 * kBQ;
-      const float* dd = l2 + kBQ;
+      // dS^T row r: 64 bf16 = eight 16-byte chunks, 128-byte swizzle (chunk c at c ^ (r & 7))
+      uint8_t* ds_row = smem + S::kDS + bi * S::kDSBytes + r * 128;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sr[32], dr[32], pk[16], dk[16];
-        tmem_ld32(tS + lane_addr + cc * 32, sr);
-        tmem_ld32(tdP + lane_addr + cc * 32, dr);
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2], dsv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qc = cc * 32 + c + u;
-            const int64_t q = q0 + qc;
-            float pr = ex2(__uint_as_float(sr[c + u]) * p.scale_log2 - l2[qc]);
-            if (partial && ((lts <= q && q < lte) || (uts <= q && q < ute))) pr = 0.f;
-            pv[u] = pr;
-            dsv[u] = pr * (__uint_as_float(dr[c + u]) - dd[qc]);
-          }
-          pk[c >> 1] = pack_bf16(pv[0], pv[1]);
-          dk[c >> 1] = pack_bf16(dsv[0], dsv[1]);
-        }
-        // P^T (bf16 pairs) over S^T columns [16 cc, 16 cc + 16): S^T columns >= 32 cc + 32 are still unread
-        tmem_st16(tS + lane_addr + cc * 16, pk);
-        // dS^T row r, queries [32 cc, 32 cc + 32): four 16-byte chunks, 128-byte swizzle (chunk c at c ^ (r & 7))
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int chunk = cc * 4 + c;
-          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
-        }
-      }
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) =
+            make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(S::DS_READY));
@@ -281,26 +304,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q * D;
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
-      const int ent = ld_nc_i32(entries + (i >> 1));
-      const int q0 = (ent >> 1) * kTile + (i & 1) * kBQ;
+      const int q0 = sub_q0(i);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DQ_FULL), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t a0[32], a1[32];
-      tmem_ld32(tdQ + lane_addr, a0);
-      tmem_ld32(tdQ + lane_addr + 32, a1);
+      uint32_t a[64];
+      tmem_ld64(tdQ + lane_addr, a);
       tc_fence_before();
       mbar_arrive(bar(S::DQ_EMPTY));
       if (d < D) {
         float* blk = acc_bh + (int64_t)q0 * D;  // [16 groups of 4 queries][D][4]
 #pragma unroll
-        for (int g = 0; g < 8; ++g)
-          red_add_v4(blk + (g * D + d) * 4, __uint_as_float(a0[4 * g]), __uint_as_float(a0[4 * g + 1]),
-                     __uint_as_float(a0[4 * g + 2]), __uint_as_float(a0[4 * g + 3]));
-#pragma unroll
-        for (int g = 0; g < 8; ++g)
-          red_add_v4(blk + ((g + 8) * D + d) * 4, __uint_as_float(a1[4 * g]), __uint_as_float(a1[4 * g + 1]),
-                     __uint_as_float(a1[4 * g + 2]), __uint_as_float(a1[4 * g + 3]));
+        for (int g = 0; g < 16; ++g)
+          red_add_v4(blk + (g * D + d) * 4, __uint_as_float(a[4 * g]), __uint_as_float(a[4 * g + 1]),
+                     __uint_as_float(a[4 * g + 2]), __uint_as_float(a[4 * g + 3]));
       }
     }
     if (!ok) record_failure(p.status, abort_flag, 14);
@@ -386,28 +403,33 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
   for (int64_t k = t; k < n4; k += (int64_t)gridDim.x * blockDim.x) a4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ[b, i, h, :] = scale * acc (accumulator layout [B,H,n_q/64][16][D][4]); 8 d per thread.
+// dQ[b, i, h, :] = scale * acc for one 64-row block per CTA: the block (a
+// contiguous 16 x D x 4 fp32 run) is read coalesced into shared memory (padded
+// against bank conflicts), then each thread writes 8 consecutive d of one row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
                                                      int B, int H, int n_q, float scale) {
-  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)B * n_q * H * (D / 8);
-  if (t >= total) return;
-  const int d0 = (int)(t % (D / 8)) * 8;
-  const int64_t row = t / (D / 8);  // (b, i, h) in output order
-  const int h = (int)(row % H);
-  const int64_t bi = row / H;
-  const int i = (int)(bi % n_q), b = (int)(bi / n_q);
-  const float* blk = acc + (((int64_t)b * H + h) * n_q + (i & ~63)) * D;
-  const int g = (i & 63) >> 2, u = i & 3;
-  uint32_t w[4];
+  __shared__ float4 buf[16 * D + 2 * D];  // one float4 of padding per 8
+  const int blocks_per_bh = n_q / 64;
+  const int64_t bh = blockIdx.x / blocks_per_bh;
+  const int qb = blockIdx.x % blocks_per_bh;
+  const int b = (int)(bh / H), h = (int)(bh % H);
+  const float4* src = reinterpret_cast<const float4*>(acc + (bh * n_q + (int64_t)qb * 64) * D);
+  for (int k = threadIdx.x; k < 16 * D; k += blockDim.x) buf[k + (k >> 3)] = __ldg(src + k);
+  __syncthreads();
+  for (int w = threadIdx.x; w < 64 * (D / 8); w += blockDim.x) {
+    const int q = w / (D / 8), d0 = (w % (D / 8)) * 8;
+    const int g = q >> 2, u = q & 3;
+    float x[8];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const float x0 = __ldg(blk + (g * D + d0 + 2 * c) * 4 + u) * scale;
-    const float x1 = __ldg(blk + (g * D + d0 + 2 * c + 1) * 4 + u) * scale;
-    w[c] = pack_bf16(x0, x1);
+    for (int c = 0; c < 8; ++c) {
+      const int k = g * D + d0 + c;
+      const float4 f = buf[k + (k >> 3)];
+      x[c] = (u == 0 ? f.x : u == 1 ? f.y : u == 2 ? f.z : f.w) * scale;
+    }
+    __nv_bfloat16* row = dq + (((int64_t)b * n_q + (int64_t)qb * 64 + q) * H + h) * D + d0;
+    st_global_v4(row, pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
   }
-  st_global_v4(dq + row * D + d0, w[0], w[1], w[2], w[3]);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -468,9 +490,8 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   if (cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) != cudaSuccess)
     return FM_ERR_CUDA;
   bwd_kernel<D><<<dim3(p.T_k, p.H, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, p);
-  const int64_t cvt = rows * (D / 8);
-  bwd_dq_kernel<D><<<(unsigned)((cvt + 255) / 256), 256, 0, stream>>>(acc, static_cast<__nv_bfloat16*>(dq), a->B,
-                                                                       a->H, a->n_q, a->scale);
+  bwd_dq_kernel<D><<<(unsigned)((int64_t)a->B * a->H * (a->n_q / 64)), 256, 0, stream>>>(
+      acc, static_cast<__nv_bfloat16*>(dq), a->B, a->H, a->n_q, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

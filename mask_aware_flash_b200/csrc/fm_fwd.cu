@@ -444,7 +444,7 @@ fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const
   if (a->dtype != 0) return FM_ERR_UNSUPPORTED;
   if (a->D != 64 && a->D != 128) return FM_ERR_UNSUPPORTED;
   if (a->n_q % kTile || a->n_k % kTile) return FM_ERR_UNSUPPORTED;
-  if (a->n_k / kTile > kMaxList) return FM_ERR_UNSUPPORTED;
+  if (a->n_k / kTile > kMaxList || a->n_q / kTile > kMaxList) return FM_ERR_UNSUPPORTED;  // lists held in smem
   if (!a->q || !a->k || !a->v) return FM_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->k) | reinterpret_cast<uintptr_t>(a->v)) & 15)
     return FM_ERR_INVALID_ARG;

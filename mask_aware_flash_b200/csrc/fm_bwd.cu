@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   using S = BwdSmem<D>;
   constexpr int NS = S::kQStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = (int)blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -258,27 +258,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       const float4* l2 = reinterpret_cast<const float4*>(stats + st * 2 * kBQ);
       const float4* dd = l2 + kBQ / 4;
+      // row-interval test (partial tiles only) as a 64-bit mask of this key's masked queries
+      uint64_t mbits = 0;
+      if (partial) {
+#pragma unroll
+        for (int qc = 0; qc < kBQ; ++qc) {
+          const int64_t q = q0 + qc;
+          mbits |= (uint64_t)(((lts <= q && q < lte) || (uts <= q && q < ute)) ? 1u : 0u) << qc;
+        }
+      }
+      const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
       uint32_t pk[32], dk[32];
 #pragma unroll
       for (int c4 = 0; c4 < kBQ / 4; ++c4) {
         const float4 L = l2[c4], Dd = dd[c4];
-        const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {Dd.x, Dd.y, Dd.z, Dd.w};
-        float pv[4], dsv[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int qc = c4 * 4 + u;
-          float pr = ex2(fmaf(__uint_as_float(sd[qc]), p.scale_log2, -lv[u]));  // 0 on empty rows (lse2 = +inf)
-          if (partial) {
-            const int64_t q = q0 + qc;
-            if ((lts <= q && q < lte) || (uts <= q && q < ute)) pr = 0.f;
-          }
-          pv[u] = pr;
-          dsv[u] = pr * (__uint_as_float(sd[64 + qc]) - dv[u]);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int qc = c4 * 4 + 2 * h2;
+          const uint64_t nl2 = h2 ? f2pack(-L.z, -L.w) : f2pack(-L.x, -L.y);
+          const uint64_t nd2 = h2 ? f2pack(-Dd.z, -Dd.w) : f2pack(-Dd.x, -Dd.y);
+          const uint64_t x2 = fma2(((uint64_t)sd[qc + 1] << 32) | sd[qc], sc2, nl2);
+          float p0 = ex2(f2lo(x2)), p1 = ex2(f2hi(x2));  // 0 on empty rows (lse2 = +inf)
+          p0 = ((mbits >> qc) & 1) ? 0.f : p0;
+          p1 = ((mbits >> (qc + 1)) & 1) ? 0.f : p1;
+          const uint64_t pp = f2pack(p0, p1);
+          const uint64_t ds2 = mul2(pp, add2(((uint64_t)sd[64 + qc + 1] << 32) | sd[64 + qc], nd2));
+          pk[qc >> 1] = pack_bf16(p0, p1);
+          dk[qc >> 1] = pack_bf16(f2lo(ds2), f2hi(ds2));
         }
-        pk[2 * c4] = pack_bf16(pv[0], pv[1]);
-        pk[2 * c4 + 1] = pack_bf16(pv[2], pv[3]);
-        dk[2 * c4] = pack_bf16(dsv[0], dsv[1]);
-        dk[2 * c4 + 1] = pack_bf16(dsv[2], dsv[3]);
       }
       // P^T (bf16 pairs) over this buffer's first 32 S^T columns (all S^T values are in registers)
       tmem_st32(tmem + bi * 64 + lane_addr, pk);

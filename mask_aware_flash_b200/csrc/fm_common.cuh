@@ -267,6 +267,44 @@ __device__ __forceinline__ float ex2(float x) {  // 2^x on the MUFU unit (ftz)
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Base of the dynamic shared memory rounded up to 1024 bytes, staying a shared-space
+// pointer (so accesses through it compile to shared loads and stores).
+__device__ __forceinline__ uint8_t* smem_base_1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
+// packed fp32 pairs (sm_100 f32x2 arithmetic); .x is the low half
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// acc + (both bf16 halves of w), fp32 accumulate (mixed-precision adds)
+__device__ __forceinline__ float add_bf16x2_to_f32(uint32_t w, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 %0, lo, %2;\n\t"
+      "add.rn.f32.bf16 %0, hi, %0;\n\t}"
+      : "=f"(r) : "r"(w), "f"(acc));
+  return r;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {  // three-input max (sm_100)
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using S = FwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = p.n_pairs - 1 - (int)blockIdx.x;  // long (late causal) query tiles first
   const int h = blockIdx.y, b = blockIdx.z;
@@ -305,34 +305,43 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             s[c] = msk ? __float_as_uint(kNegInf) : s[c];
           }
         }
-        float mx0 = kNegInf, mx1 = kNegInf;
+        // row maximum: four independent three-input max chains
+        float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
-        for (int c = 0; c < kTile; c += 4) {
-          mx0 = fmax3(mx0, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-          mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        for (int c = 0; c < kTile; c += 8) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            mx[u] = fmax3(mx[u], __uint_as_float(s[c + 2 * u]), __uint_as_float(s[c + 2 * u + 1]));
         }
-        const float m_tile = fmaxf(mx0, mx1) * p.scale_log2;
+        const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
         // move the running maximum only when it grows by more than the threshold
         const bool move = (m_tile - m_run) > kRescaleThreshold;  // false when both are -inf
         const float m_new = move ? m_tile : m_run;
         const float alpha = move ? ex2(m_run - m_new) : 1.f;
         const float m_use = (m_new == kNegInf) ? 0.f : m_new;
-        // rs: exact fp32 row sum (LSE); rq: sum of the bf16-rounded P the PV product
-        // actually uses (O is normalised by it, so O stays a convex combination of V rows)
-        float rs = 0.f, rq = 0.f;
+        // P = 2^(s*scale - m) on pairs (f32x2); rs: exact fp32 row sum (LSE); rq: sum of
+        // the bf16-rounded P the PV product uses (O is normalised by it, so O stays a
+        // convex combination of V rows).  Independent accumulators break the add chains.
+        const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-m_use, -m_use);
+        uint64_t rs2[4] = {0, 0, 0, 0};
+        float rq[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < kTile; c += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[c]), p.scale_log2, -m_use));
-          const float p1 = ex2(fmaf(__uint_as_float(s[c + 1]), p.scale_log2, -m_use));
-          rs += p0 + p1;
+          const uint64_t x2 = fma2(((uint64_t)s[c + 1] << 32) | s[c], sc2, nm2);
+          const float p0 = ex2(f2lo(x2)), p1 = ex2(f2hi(x2));
+          const int k = (c >> 1) & 3;
+          rs2[k] = add2(rs2[k], f2pack(p0, p1));
           const uint32_t w = pack_bf16(p0, p1);
-          rq += bf16_lo(w) + bf16_hi(w);
+          rq[k] = add_bf16x2_to_f32(w, rq[k]);
           pk[c >> 1] = w;
         }
+        const uint64_t rs2a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
+        const float rs = f2lo(rs2a) + f2hi(rs2a);
+        const float rqs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
         tmem_st64(tS, pk);
         l_run = l_run * alpha + rs;
-        lq_run = lq_run * alpha + rq;
+        lq_run = lq_run * alpha + rqs;
         m_run = m_new;
         if (__any_sync(0xffffffffu, move && j > 0)) {
           // O holds the sum over earlier tiles: wait for the last PV, rescale in TMEM

@@ -30,7 +30,7 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kBQ = 64;  // query rows per backward sub-tile
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 448;  // 2 x compute, 1 x dQ drain warpgroups, load warp, MMA warp
 constexpr int kMaxList = 4096;  // query tiles per key tile held in shared memory
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kPosInf = __builtin_huge_valf();
@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < S::kNumBars; ++k) mbar_init(bar(k), 1);
-    mbar_init(bar(S::DP_FREE), kTile);
-    mbar_init(bar(S::DS_READY), kTile);
+    mbar_init(bar(S::DP_FREE), 2 * kTile);
+    mbar_init(bar(S::DS_READY), 2 * kTile);
     mbar_init(bar(S::DQ_EMPTY), kTile);
     *abort_flag = 0;
     misc[2] = 0;
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int t = threadIdx.x; t < kTile * 64 * 2 / 16; t += blockDim.x) z[t] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(misc), 512);
     tmem_relinquish();
   }
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tdP = tmem + 128, tdQ = tmem + 192, tdV = tmem + 256, tdK = tmem + 384;
   auto sub_q0 = [&](int i) { return (int)(list[i >> 1] >> 1) * kTile + (i & 1) * kBQ; };
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ load role
     if (lane == 0 && cnt > 0) {
       prefetch_tmap(&tm_q);
@@ -153,26 +153,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bulk_load(smem_u32(stats + st * 2 * kBQ + kBQ), p.dvec + bh * p.n_q + q0, kBQ * 4, fb);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------- MMA role
     if (lane == 0 && cnt > 0) {
       constexpr uint32_t kIdSdp = idesc_bf16(128, kBQ, false, false);  // S^T, dP^T: [key][q]
       constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);     // dV, dK: [key][d], B MN-major
       constexpr uint32_t kIdDq = idesc_bf16(128, kBQ, true, true);     // dQ^T: [d][q], A and B MN-major
+      // descriptor words (128-byte swizzle, SBO = 8 rows x 128 B); per k-step only the low word moves
+      constexpr uint32_t kHi = desc_hi(1024);
+      constexpr uint32_t kStageW = S::kQStage >> 4, kDSW = S::kDSBytes >> 4;
+      const uint32_t lo_k = desc_lo(k_s, 16), lo_v = desc_lo(v_s, 16);           // K-major A of S^T, dP^T
+      const uint32_t lo_kt = desc_lo(k_s, 16384);                                  // K^T as MN-major A of dQ^T
+      const uint32_t lo_q = desc_lo(q_s, 16), lo_do = desc_lo(do_s, 16);         // K-major B of S^T, dP^T
+      const uint32_t lo_qmn = desc_lo(q_s, 8192), lo_domn = desc_lo(do_s, 8192);  // MN-major B of dK, dV
+      const uint32_t lo_ds = desc_lo(ds_s, 16), lo_dsmn = desc_lo(ds_s, 16384);   // dS^T as A of dK / B of dQ^T
       auto issue_s = [&](int i) {  // S^T_i = K Q_i^T
-        const uint32_t qs = q_s + (i % NS) * S::kQStage, tS = tmem + (i & 1) * 64;
+        const uint32_t qa = lo_q + (i % NS) * kStageW, tS = tmem + (i & 1) * 64;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t okv = (k >> 2) * 16384 + (k & 3) * 32, oq = (k >> 2) * 8192 + (k & 3) * 32;
-          umma_ss(tS, smem_desc(k_s + okv, 16, 1024), smem_desc(qs + oq, 16, 1024), kIdSdp, k > 0 ? 1u : 0u);
+          const uint32_t okv = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, oq = ((k >> 2) * 8192 + (k & 3) * 32) >> 4;
+          umma_ss_w(tS, lo_k + okv, kHi, qa + oq, kHi, kIdSdp, k > 0 ? 1u : 0u);
         }
       };
       auto issue_dp = [&](int i) {  // dP^T_i = V dO_i^T
-        const uint32_t dos = do_s + (i % NS) * S::kQStage;
+        const uint32_t da = lo_do + (i % NS) * kStageW;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t okv = (k >> 2) * 16384 + (k & 3) * 32, oq = (k >> 2) * 8192 + (k & 3) * 32;
-          umma_ss(tdP, smem_desc(v_s + okv, 16, 1024), smem_desc(dos + oq, 16, 1024), kIdSdp, k > 0 ? 1u : 0u);
+          const uint32_t okv = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, oq = ((k >> 2) * 8192 + (k & 3) * 32) >> 4;
+          umma_ss_w(tdP, lo_v + okv, kHi, da + oq, kHi, kIdSdp, k > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(S::KV_FULL), 0, abort_flag) && mbar_wait(bar(S::QDO_FULL0), 0, abort_flag);
@@ -204,17 +212,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t qs = q_s + st * S::kQStage, dos = do_s + st * S::kQStage, dss = ds_s + bi * S::kDSBytes;
+        const uint32_t qmn = lo_qmn + st * kStageW, domn = lo_domn + st * kStageW;
+        const uint32_t dsa = lo_ds + bi * kDSW, dsb = lo_dsmn + bi * kDSW;
         const uint32_t tP = tmem + bi * 64;
-        // dV += P^T dO (P^T bf16 in TMEM, 16 queries = 8 columns per step; dO MN-major)
+        // dV += P^T dO (P^T bf16 in TMEM, 16 queries = 8 columns per step; dO MN-major).  Queries
+        // [0, 32) of P^T sit in columns [0, 16) of the buffer, queries [32, 64) in columns [32, 48).
 #pragma unroll
         for (int k = 0; k < kBQ / 16; ++k)
-          umma_ts(tdV, tP + k * 8, smem_desc(dos + k * 2048, 8192, 1024), kIdAcc, (i > 0 || k > 0) ? 1u : 0u);
+          umma_ts_w(tdV, tP + (k >> 1) * 32 + (k & 1) * 8, domn + ((k * 2048) >> 4), kHi, kIdAcc,
+                    (i > 0 || k > 0) ? 1u : 0u);
         // dK += dS^T Q (dS^T K-major in smem, one swizzle atom wide; Q MN-major)
 #pragma unroll
         for (int k = 0; k < kBQ / 16; ++k)
-          umma_ss(tdK, smem_desc(dss + k * 32, 16, 1024), smem_desc(qs + k * 2048, 8192, 1024), kIdAcc,
-                  (i > 0 || k > 0) ? 1u : 0u);
+          umma_ss_w(tdK, dsa + ((k * 32) >> 4), kHi, qmn + ((k * 2048) >> 4), kHi, kIdAcc, (i > 0 || k > 0) ? 1u : 0u);
         umma_commit(bar(S::QDO_EMPTY0 + st));
         if (i > 0 && !mbar_wait(bar(S::DQ_EMPTY), (i - 1) & 1, abort_flag)) {
           ok = false;
@@ -224,8 +234,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dQ^T = K^T dS^T (K^T: M = d, MN-major; dS^T as B: N = q, MN-major; 16 keys per step)
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          umma_ss(tdQ, smem_desc(k_s + k * 2048, 16384, 1024), smem_desc(dss + k * 2048, 16384, 1024), kIdDq,
-                  k > 0 ? 1u : 0u);
+          umma_ss_w(tdQ, lo_kt + ((k * 2048) >> 4), kHi, dsb + ((k * 2048) >> 4), kHi, kIdDq, k > 0 ? 1u : 0u);
         umma_commit(bar(S::DQ_FULL));
         umma_commit(bar(S::DS_EMPTY0 + bi));
       }
@@ -234,43 +243,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       umma_commit(bar(S::DRAIN));
       mbar_wait(bar(S::DRAIN), 0, never);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------ P^T / dS^T role (row = key)
-    const int r = threadIdx.x;
+  } else if (warp < 8) {
+    // ---------------------------- P^T / dS^T role (row = key), warps 0-7
+    // Warpgroup hf handles queries [32 hf, 32 hf + 32) of every 64-query sub-tile.
+    const int hf = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const int c0 = 32 * hf;
     const int64_t j = (int64_t)kt * kTile + r;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const int64_t voff = bhm * p.n_k + j;
     const int32_t lts = p.vec[0] ? __ldg(p.vec[0] + voff) : p.n_q, lte = p.vec[1] ? __ldg(p.vec[1] + voff) : p.n_q;
     const int32_t uts = p.vec[2] ? __ldg(p.vec[2] + voff) : 0, ute = p.vec[3] ? __ldg(p.vec[3] + voff) : 0;
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
       const int st = i % NS, bi = i & 1;
-      const int q0 = sub_q0(i);
+      const int q0 = sub_q0(i) + c0;
       const bool partial = list[i >> 1] & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(S::SDP_FULL), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sd[128];  // [0, 64): S^T row, [64, 128): dP^T row
-      tmem_ld64x2(tmem + bi * 64 + lane_addr, tdP + lane_addr, sd);
+      uint32_t sd[64];  // [0, 32): S^T row, [32, 64): dP^T row (this warpgroup's queries)
+      tmem_ld32x2(tmem + bi * 64 + c0 + lane_addr, tdP + c0 + lane_addr, sd);
       tc_fence_before();
       mbar_arrive(bar(S::DP_FREE));  // dP^T columns may be overwritten by the next sub-tile
       ok = __all_sync(0xffffffffu, mbar_wait(bar(S::QDO_FULL0 + st), (i / NS) & 1, abort_flag));
       if (!ok) break;
-      const float4* l2 = reinterpret_cast<const float4*>(stats + st * 2 * kBQ);
-      const float4* dd = l2 + kBQ / 4;
-      // row-interval test (partial tiles only) as a 64-bit mask of this key's masked queries
-      uint64_t mbits = 0;
+      const float4* l2 = reinterpret_cast<const float4*>(stats + st * 2 * kBQ + c0);
+      const float4* dd = reinterpret_cast<const float4*>(stats + st * 2 * kBQ + kBQ + c0);
+      // row-interval test (partial tiles only) as a mask of this key's masked queries
+      uint32_t mbits = 0;
       if (partial) {
 #pragma unroll
-        for (int qc = 0; qc < kBQ; ++qc) {
+        for (int qc = 0; qc < 32; ++qc) {
           const int64_t q = q0 + qc;
-          mbits |= (uint64_t)(((lts <= q && q < lte) || (uts <= q && q < ute)) ? 1u : 0u) << qc;
+          mbits |= (((lts <= q && q < lte) || (uts <= q && q < ute)) ? 1u : 0u) << qc;
         }
       }
       const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
-      uint32_t pk[32], dk[32];
+      uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int c4 = 0; c4 < kBQ / 4; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {
         const float4 L = l2[c4], Dd = dd[c4];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -281,32 +293,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           float p0 = ex2(f2lo(x2)), p1 = ex2(f2hi(x2));  // 0 on empty rows (lse2 = +inf)
           p0 = ((mbits >> qc) & 1) ? 0.f : p0;
           p1 = ((mbits >> (qc + 1)) & 1) ? 0.f : p1;
-          const uint64_t pp = f2pack(p0, p1);
-          const uint64_t ds2 = mul2(pp, add2(((uint64_t)sd[64 + qc + 1] << 32) | sd[64 + qc], nd2));
+          const uint64_t ds2 = mul2(f2pack(p0, p1), add2(((uint64_t)sd[32 + qc + 1] << 32) | sd[32 + qc], nd2));
           pk[qc >> 1] = pack_bf16(p0, p1);
           dk[qc >> 1] = pack_bf16(f2lo(ds2), f2hi(ds2));
         }
       }
-      // P^T (bf16 pairs) over this buffer's first 32 S^T columns (all S^T values are in registers)
-      tmem_st32(tmem + bi * 64 + lane_addr, pk);
+      // P^T (bf16 pairs) into 16 columns of this warpgroup's own S^T range (already read)
+      tmem_st16(tmem + bi * 64 + c0 + lane_addr, pk);
       if (i >= 2) {  // dS^T buffer bi free: the dK / dQ^T MMAs of sub-tile i-2 have read it
         ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DS_EMPTY0 + bi), ((i >> 1) - 1) & 1, abort_flag));
         if (!ok) break;
       }
-      // dS^T row r: 64 bf16 = eight 16-byte chunks, 128-byte swizzle (chunk c at c ^ (r & 7))
+      // dS^T row r, queries [c0, c0+32): four 16-byte chunks, 128-byte swizzle (chunk c at c ^ (r & 7))
       uint8_t* ds_row = smem + S::kDS + bi * S::kDSBytes + r * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) =
+      for (int c = 0; c < 4; ++c) {
+        const int chunk = 4 * hf + c;
+        *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
             make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(S::DS_READY));
     }
     if (!ok) record_failure(p.status, abort_flag, 13);
   } else {
-    // ------------------------------------- dQ drain role (row = d), warps 4-7
-    const int d = threadIdx.x - 128;
+    // ------------------------------------- dQ drain role (row = d), warps 8-11
+    const int d = threadIdx.x - 256;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q * D;
     bool ok = true;
@@ -364,7 +377,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

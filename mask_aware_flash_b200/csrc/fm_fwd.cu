@@ -196,21 +196,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool has_cur = ok && it.next(kt, c0, c1);
       int np[2] = {0, 0};  // P tiles consumed per query tile (p_full phases)
       bool acc[2] = {false, false};
+      // descriptor words: 128-byte swizzle, SBO = 8 rows x 128 B; per k-step only the low word moves
+      constexpr uint32_t kHi = desc_hi(1024);
+      const uint32_t lo_q = desc_lo(q_s, 16), lo_k = desc_lo(k_s, 16), lo_v = desc_lo(v_s, 16384);
+      constexpr uint32_t kTileW = S::kTileBytes >> 4;  // one tile, in 16-byte descriptor units
+      auto issue_s = [&](int t, int kslot) {  // S_t = Q_t K^T
+        const uint32_t qa = lo_q + t * kTileW, ka = lo_k + kslot * kTileW;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;  // swizzle-atom column, 16-element K step
+          umma_ss_w(tmem + t * 256, qa + off, kHi, ka + off, kHi, kIdescQK, k > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(S::S_FULL0 + t));
+      };
       if (has_cur) {
         ok = mbar_wait(bar(S::K_FULL0), 0, abort_flag);
         if (ok) {
           tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (t ? c1 : c0) {
-              const uint32_t qa = q_s + t * S::kTileBytes, ka = k_s;
-#pragma unroll
-              for (int k = 0; k < D / 16; ++k) {
-                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                umma_ss(tmem + t * 256, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), kIdescQK,
-                        k > 0 ? 1u : 0u);
-              }
-              umma_commit(bar(S::S_FULL0 + t));
-            }
+          if (c0) issue_s(0, 0);
+          if (c1) issue_s(1, 0);
           umma_commit(bar(S::K_EMPTY0));
         }
       }
@@ -235,21 +239,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             ++np[t];
             tc_fence_after();
-            const uint32_t va = v_s + slot * S::kTileBytes;
+            const uint32_t va = lo_v + slot * kTileW;
 #pragma unroll
             for (int k = 0; k < kTile / 16; ++k)  // 16 kv rows per step; P columns advance 8 (bf16 pairs)
-              umma_ts(tO, tS + k * 8, smem_desc(va + k * 2048, 16384, 1024), kIdescPV, (acc[t] || k > 0) ? 1u : 0u);
+              umma_ts_w(tO, tS + k * 8, va + ((k * 2048) >> 4), kHi, kIdescPV, (acc[t] || k > 0) ? 1u : 0u);
             umma_commit(bar(S::O_DONE0 + t));
             acc[t] = true;
           }
           if (has_next && (t ? n1c : n0c)) {  // S_t = Q_t K(e+1)^T, after PV_t(e) has read P_t
-            const uint32_t qa = q_s + t * S::kTileBytes, ka = k_s + nslot * S::kTileBytes;
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-              umma_ss(tS, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
-            }
-            umma_commit(bar(S::S_FULL0 + t));
+            tc_fence_after();
+            issue_s(t, nslot);
           }
         }
         if (!ok) break;

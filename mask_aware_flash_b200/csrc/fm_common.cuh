@@ -346,6 +346,29 @@ __device__ __forceinline__ float add_bf16x2_to_f32(uint32_t w, float acc) {
   return r;
 }
 
+// 2^x for a pair of fp32 values on the FMA / integer pipes (the MUFU unit's ex2
+// is the co-bottleneck of the forward softmax).  Argument reduction: n = round(x)
+// by adding and subtracting 1.5 * 2^23 (round-to-nearest in fp32), f = x - n in
+// [-1/2, 1/2]; 2^f by the degree-3 minimax polynomial (relative error 7.5e-5)
+// that a Remez exchange fits in mask_aware_flash_b200/exp2_poly.py; 2^n is added
+// to the exponent field.  x is clamped at -125 so the exponent never leaves the
+// normal range: inputs below that (masked scores are -inf) give about 2^-125.
+constexpr float kExp2C0 = 9.999280572e-01f, kExp2C1 = 6.932609677e-01f, kExp2C2 = 2.426111251e-01f,
+                kExp2C3 = 5.517166853e-02f;
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t xc = f2pack(fmaxf(f2lo(x2), -125.f), fmaxf(f2hi(x2), -125.f));
+  const uint64_t t2 = add2(xc, f2pack(kRound, kRound));          // low mantissa bits hold n
+  const uint64_t r2 = add2(t2, f2pack(-kRound, -kRound));        // n as fp32
+  const uint64_t f2 = fma2(r2, f2pack(-1.f, -1.f), xc);          // f = x - n
+  uint64_t q2 = fma2(f2, f2pack(kExp2C3, kExp2C3), f2pack(kExp2C2, kExp2C2));
+  q2 = fma2(q2, f2, f2pack(kExp2C1, kExp2C1));
+  q2 = fma2(q2, f2, f2pack(kExp2C0, kExp2C0));
+  const uint32_t lo = (uint32_t)q2 + ((uint32_t)t2 << 23);
+  const uint32_t hi = (uint32_t)(q2 >> 32) + ((uint32_t)(t2 >> 32) << 23);
+  return ((uint64_t)hi << 32) | lo;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {  // three-input max (sm_100)
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -36,6 +36,8 @@ constexpr int kFwdThreads = 320;
 constexpr int kMaxList = 4096;  // key tiles per query tile held in shared memory (n_k <= 524288)
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
+constexpr int kPolyEvery = 4;  // one score pair in kPolyEvery takes exp2_poly2 instead of MUFU ex2
+constexpr float kLiveSum = 1e-20f;  // a live row's sum is >= ~1; masked scores add ~2^-125 each
 
 struct FwdParams {
   const int32_t* row_count;    // [B, Hm, T_q]
@@ -58,7 +60,8 @@ struct FwdSmem {
   static constexpr int kList = kMask + 2 * 4 * kTile * 4;  // two row lists, kMaxList uint16 each
   static constexpr int kBar = kList + 2 * kMaxList * 2;
   enum { Q_FULL, K_FULL0, K_FULL1, K_EMPTY0, K_EMPTY1, V_FULL0, V_FULL1, V_EMPTY0, V_EMPTY1, S_FULL0, S_FULL1,
-         P_FULL0, P_FULL1, O_DONE0, O_DONE1, M_FULL0, M_FULL1, M_EMPTY0, M_EMPTY1, DRAIN, kNumBars };
+         P_FULL0, P_FULL1, P_HALF0, P_HALF1, O_DONE0, O_DONE1, M_FULL0, M_FULL1, M_EMPTY0, M_EMPTY1, DRAIN,
+         kNumBars };
   static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag, [2] zero
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;       // slack for 1024-byte alignment of the base
@@ -117,6 +120,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int k = 0; k < S::kNumBars; ++k) mbar_init(bar(k), 1);
     mbar_init(bar(S::P_FULL0), kTile);
     mbar_init(bar(S::P_FULL1), kTile);
+    mbar_init(bar(S::P_HALF0), kTile);
+    mbar_init(bar(S::P_HALF1), kTile);
     mbar_init(bar(S::M_EMPTY0), 2 * kTile);
     mbar_init(bar(S::M_EMPTY1), 2 * kTile);
     *abort_flag = 0;
@@ -232,17 +237,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const uint32_t tS = tmem + t * 256, tO = tS + 128;
-          if (t ? c1 : c0) {  // O_t += P_t V(e)
+          if (t ? c1 : c0) {  // O_t += P_t V(e): first half of P as soon as it is in TMEM
+            if (!mbar_wait(bar(S::P_HALF0 + t), np[t] & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t va = lo_v + slot * kTileW;
+#pragma unroll
+            for (int k = 0; k < kTile / 32; ++k)  // 16 kv rows per step; P columns advance 8 (bf16 pairs)
+              umma_ts_w(tO, tS + k * 8, va + ((k * 2048) >> 4), kHi, kIdescPV, (acc[t] || k > 0) ? 1u : 0u);
             if (!mbar_wait(bar(S::P_FULL0 + t), np[t] & 1, abort_flag)) {
               ok = false;
               break;
             }
             ++np[t];
             tc_fence_after();
-            const uint32_t va = lo_v + slot * kTileW;
 #pragma unroll
-            for (int k = 0; k < kTile / 16; ++k)  // 16 kv rows per step; P columns advance 8 (bf16 pairs)
-              umma_ts_w(tO, tS + k * 8, va + ((k * 2048) >> 4), kHi, kIdescPV, (acc[t] || k > 0) ? 1u : 0u);
+            for (int k = kTile / 32; k < kTile / 16; ++k)
+              umma_ts_w(tO, tS + k * 8, va + ((k * 2048) >> 4), kHi, kIdescPV, 1u);
             umma_commit(bar(S::O_DONE0 + t));
             acc[t] = true;
           }
@@ -318,46 +331,62 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float m_new = move ? m_tile : m_run;
         const float alpha = move ? ex2(m_run - m_new) : 1.f;
         const float m_use = (m_new == kNegInf) ? 0.f : m_new;
-        // P = 2^(s*scale - m) on pairs (f32x2); rs: exact fp32 row sum (LSE); rq: sum of
-        // the bf16-rounded P the PV product uses (O is normalised by it, so O stays a
-        // convex combination of V rows).  Independent accumulators break the add chains.
+        // P = 2^(s*scale - m) on pairs (f32x2), in two halves of 64 scores: each half is
+        // stored (bf16 pairs over the first S columns) and published on its own barrier so
+        // the PV product starts on the first half while the second is computed.
+        // rs: exact fp32 row sum (LSE); rq: sum of the bf16-rounded P the PV product uses
+        // (O is normalised by it, so O stays a convex combination of V rows).
         const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-m_use, -m_use);
         uint64_t rs2[4] = {0, 0, 0, 0};
         float rq[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[64];
 #pragma unroll
-        for (int c = 0; c < kTile; c += 2) {
-          const uint64_t x2 = fma2(((uint64_t)s[c + 1] << 32) | s[c], sc2, nm2);
-          const float p0 = ex2(f2lo(x2)), p1 = ex2(f2hi(x2));
-          const int k = (c >> 1) & 3;
-          rs2[k] = add2(rs2[k], f2pack(p0, p1));
-          const uint32_t w = pack_bf16(p0, p1);
-          rq[k] = add_bf16x2_to_f32(w, rq[k]);
-          pk[c >> 1] = w;
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < kTile / 2; c += 2) {
+            const int cs = hh * (kTile / 2) + c;
+            const uint64_t x2 = fma2(((uint64_t)s[cs + 1] << 32) | s[cs], sc2, nm2);
+            float p0, p1;
+            if (((c >> 1) & (kPolyEvery - 1)) == kPolyEvery - 1) {  // this pair on the FMA pipe
+              const uint64_t e2 = exp2_poly2(x2);
+              p0 = f2lo(e2);
+              p1 = f2hi(e2);
+            } else {  // MUFU
+              p0 = ex2(f2lo(x2));
+              p1 = ex2(f2hi(x2));
+            }
+            const int k = (c >> 1) & 3;
+            rs2[k] = add2(rs2[k], f2pack(p0, p1));
+            const uint32_t w = pack_bf16(p0, p1);
+            rq[k] = add_bf16x2_to_f32(w, rq[k]);
+            pk[c >> 1] = w;
+          }
+          if (hh == 0 && __any_sync(0xffffffffu, move && j > 0)) {
+            // O holds the sum over earlier tiles: wait for the last PV, rescale it in TMEM
+            // before this tile's PV accumulates into it
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE0 + t), (j - 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < D / 16; ++cc) {
+              uint32_t orr[16];
+              tmem_ld16(tO + cc * 16, orr);
+#pragma unroll
+              for (int c = 0; c < 16; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+              tmem_st16(tO + cc * 16, orr);
+            }
+          }
+          tmem_st32(tS + hh * 32, pk);
+          tc_fence_before();
+          mbar_arrive(bar((hh ? S::P_FULL0 : S::P_HALF0) + t));
         }
+        if (!ok) break;
         const uint64_t rs2a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
         const float rs = f2lo(rs2a) + f2hi(rs2a);
         const float rqs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
-        tmem_st64(tS, pk);
         l_run = l_run * alpha + rs;
         lq_run = lq_run * alpha + rqs;
         m_run = m_new;
-        if (__any_sync(0xffffffffu, move && j > 0)) {
-          // O holds the sum over earlier tiles: wait for the last PV, rescale in TMEM
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE0 + t), (j - 1) & 1, abort_flag));
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t orr[32];
-            tmem_ld32(tO + cc * 32, orr);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
-            tmem_st32(tO + cc * 32, orr);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bar(S::P_FULL0 + t));
         ++j;
       } else if (has_mask) {
         // keep the two warpgroups in step on the shared mask buffers
@@ -373,14 +402,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // epilogue: O = O / l, LSE = (m + log2 l) ln 2; empty rows: O = 0, LSE = -inf
     if (live_tile) {
       __nv_bfloat16* orow = p.o + (((int64_t)b * p.n_q + i) * p.H + h) * D;
-      const bool live = ok && j > 0 && l_run > 0.f;
+      const bool live = ok && j > 0 && l_run > kLiveSum;
       bool have_o = false;
       if (ok && j > 0) {
         have_o = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE0 + t), (j - 1) & 1, abort_flag));
         if (!have_o) record_failure(p.status, abort_flag, 6);
         tc_fence_after();
       }
-      const float inv = live && lq_run > 0.f ? 1.f / lq_run : 0.f;
+      const float inv = live ? 1.f / lq_run : 0.f;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t orr[32];

@@ -219,6 +219,22 @@ def cpu_baseline(wl, budget_s=15.0):
                       f"effective FLOPs = 14*D*pairs"}
 
 
+# ----------------------------------------------------------------------------- ranks
+def reduce_max(values, world, device):
+    """Element-wise maximum over all ranks (device time of the slowest rank)."""
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(world, flops_per_rank_step, steps, max_ms):
+    """Whole-job throughput: every rank processes its own replica's work in the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -304,12 +320,9 @@ def run_ours(args, rank, world, local_rank):
     bwd_ms = sum(recs[s]["f1"][m].elapsed_time(recs[s]["b1"][m]) for s in range(args.steps) for m in range(nm))
     meta_ms = sum(recs[s]["m0"][m].elapsed_time(recs[s]["f0"][m]) for s in range(args.steps) for m in range(nm))
     total_ms = sum(step_ms)
-    t = torch.tensor([total_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_ms, bwd_ms = t.tolist()
+    total_ms, fwd_ms, bwd_ms = reduce_max([total_ms, fwd_ms, bwd_ms], world, dev)
     steps = args.steps
-    value = world * (flops_fwd + flops_bwd) * steps / (total_ms * 1e-3) / 1e12
+    value = job_tflops(world, flops_fwd + flops_bwd, steps, total_ms)
 
     # end-to-end through the public API with host buffers (H2D of inputs, D2H of results)
     e2e = None
@@ -342,10 +355,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * (flops_fwd + flops_bwd) * steps / (te.item() * 1e-3) / 1e12, "unit": UNIT,
+        (te_ms,) = reduce_max([e0.elapsed_time(e1)], world, dev)
+        e2e = {"value": job_tflops(world, flops_fwd + flops_bwd, steps, te_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     assert fm.fm_get_device_status() == 0, "device-side timeout during the bench"
 

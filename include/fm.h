@@ -25,7 +25,9 @@
  *     pointer stands for its canonical empty value (LTS = LTE = n_q, UTS = UTE = 0).
  *     Vectors are int32 [B, Hm, n_k] contiguous, Hm = 1 (shared by all heads) or H.
  *   - Tensors Q, O, dO, dQ are [B, n_q, H, D] and K, V, dK, dV are [B, n_k, H, D],
- *     contiguous, element type bf16 (dtype 0).  LSE is fp32 [B, H, n_q], natural log.
+ *     contiguous, all of one element type: bf16 (dtype 0; bf16 tensor-core products) or
+ *     fp32 (dtype 1, D = 64 only; tf32 tensor-core products, fp32 accumulation).  LSE is
+ *     fp32 [B, H, n_q], natural log.
  *   - All pointers passed to compute calls are DEVICE pointers unless a parameter
  *     says "host".  The caller owns every buffer, including workspaces; the
  *     library never allocates, frees or synchronises.  Work is enqueued on
@@ -131,7 +133,7 @@ fm_status fm_localize(int32_t B, int32_t Hm, int32_t N, const int32_t* const in[
 /* Attention problem.  q, k, v are device pointers (bf16, layouts above). */
 typedef struct {
   int32_t B, H, n_q, n_k, D;
-  int32_t dtype;  /* 0 = bf16 (the only supported type) */
+  int32_t dtype;  /* 0 = bf16, 1 = fp32 (tf32 products; D = 64 only) */
   float scale;    /* softmax scale, e.g. 1/sqrt(D) */
   const void* q;
   const void* k;
@@ -144,11 +146,12 @@ typedef struct {
  * LSE_i = ln sum_{j in U_i} exp(scale q_i.k_j); a row with U_i empty gets
  * O_i = 0 and LSE_i = -inf.  Only non-skip key tiles (meta row lists) are read;
  * the row-interval test runs on partial tiles only.
- *   a      host struct; n_q, n_k multiples of 128; D in {64, 128}; dtype 0.
+ *   a      host struct; n_q, n_k multiples of 128; D in {64, 128}; dtype 0, or 1 with D = 64;
+ *          scale > 0 and finite.
  *   meta   host struct from fm_build_mask_meta with d = {B, Hm, n_q, n_k, 128, 128}.
  *   vec[4] host array of the 4 device vector pointers meta was built from
  *          (NULL entries allowed = canonical empty); 16-byte aligned.
- *   o      device bf16 [B, n_q, H, D]; lse device fp32 [B, H, n_q].
+ *   o      device [B, n_q, H, D] of the dtype; lse device fp32 [B, H, n_q].
  * Errors: FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_CUDA.
  */
 fm_status fm_attn_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], void* o,
@@ -163,8 +166,8 @@ size_t fm_attn_bwd_workspace_bytes(const fm_attn_args* a);
  *   dV_j = sum_i P_ij dO_i, dS_ij = P_ij (dO_i.v_j - D_i),
  *   dQ_i = scale sum_j dS_ij k_j, dK_j = scale sum_i dS_ij q_i.
  * Key tiles iterate their meta column lists (non-skip query tiles only).
- *   o, lse   the forward's outputs; dout device bf16 [B, n_q, H, D].
- *   dq, dk, dv device bf16 outputs (layouts above); every element is written.
+ *   o, lse   the forward's outputs; dout device [B, n_q, H, D] of the dtype.
+ *   dq, dk, dv device outputs of the dtype (layouts above); every element is written.
  *   ws       device workspace, ws_bytes >= fm_attn_bwd_workspace_bytes(a), 256-byte
  *            aligned; holds the fp32 dQ accumulator and per-row statistics.
  * Errors: FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA.

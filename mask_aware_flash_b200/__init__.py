@@ -169,11 +169,13 @@ def fm_localize(vecs, chunk_start, chunk_len, stream=None):
 
 def _args(q, k, v, scale) -> AttnArgs:
     B, n_q, H, D = q.shape
-    return AttnArgs(B, H, n_q, k.shape[1], D, 0, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr())
+    dtype = 1 if q.dtype == torch.float32 else 0
+    return AttnArgs(B, H, n_q, k.shape[1], D, dtype, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr())
 
 
 def fm_attn_fwd(q, k, v, meta: MaskMeta, vecs, scale, o=None, lse=None, stream=None):
-    """q [B, n_q, H, D], k/v [B, n_k, H, D] bf16 CUDA tensors -> o (bf16), lse [B, H, n_q] fp32."""
+    """q [B, n_q, H, D], k/v [B, n_k, H, D] CUDA tensors (bf16, or fp32 with D=64) -> o (same dtype),
+    lse [B, H, n_q] fp32."""
     B, n_q, H, D = q.shape
     if o is None:
         o = torch.empty_like(q)
@@ -192,7 +194,7 @@ def fm_attn_bwd_workspace_bytes(q, k, v, scale=1.0) -> int:
 
 def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=None, dv=None, ws=None,
                 stream=None):
-    """Gradients (bf16) of the masked attention; ws: optional uint8 CUDA workspace."""
+    """Gradients (dtype of q) of the masked attention; ws: optional uint8 CUDA workspace."""
     a = _args(q, k, v, scale)
     nbytes = lib().fm_attn_bwd_workspace_bytes(ctypes.byref(a))
     if ws is None:

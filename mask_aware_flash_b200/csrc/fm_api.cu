@@ -64,6 +64,21 @@ bool encode_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t D, uint64_
   return r == CUDA_SUCCESS;
 }
 
+// Same view of a [B, n, H, D] fp32 tensor: box (32, 1, box_rows, 1), 32 fp32 = one swizzle span.
+bool encode_tmap_f32_4d(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t n, uint64_t B,
+                        uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {D, H, n, B};
+  cuuint64_t strides[3] = {D * 4, H * D * 4, n * H * D * 4};
+  cuuint32_t box[4] = {32, 1, box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fm
 
 extern "C" {

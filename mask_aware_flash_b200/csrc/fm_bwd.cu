@@ -42,40 +42,101 @@ struct BwdParams {
   const float* lse2;           // [B, H, n_q] log2-domain LSE, +inf on empty rows
   const float* dvec;           // [B, H, n_q] D_i = dO_i . O_i
   float* dq_acc;               // [B, H, n_q/64][16][D][4] fp32
-  __nv_bfloat16* dk;           // [B, n_k, H, D]
-  __nv_bfloat16* dv;
+  void* dk;                    // [B, n_k, H, D], bf16 or fp32
+  void* dv;
   int* status;
   int B, H, Hm, n_q, n_k, T_q, T_k;
   float scale, scale_log2;
 };
 
-template <int D>
+template <int D, bool F32>
 struct BwdSmem {
-  static constexpr int kQStages = 3;
-  static constexpr int kK = 0;                       // 128 x 128 bf16 (D=64: upper half kept zero, see dQ^T)
-  static constexpr int kV = kK + kTile * 128 * 2;
-  static constexpr int kQStage = kBQ * D * 2;        // one 64-row sub-tile of Q (or dO)
-  static constexpr int kQ = kV + kTile * D * 2;      // kQStages x Q
+  static constexpr int kElem = F32 ? 4 : 2;
+  static constexpr int kQStages = F32 ? 2 : 3;       // fp32 tiles are twice as large
+  static constexpr int kDSBufs = F32 ? 1 : 2;
+  // bf16: K, 128 keys x 128 d (the d >= D part kept zero: K^T is a 128-row MMA operand for dQ^T).
+  // fp32 (D = 64): K [key][d] in the first half, K^T [d][key] (K-major, four 8 KiB atoms) in the second;
+  // V follows, so the 64 rows past the last K^T atom that a 128-row operand reads stay in bounds.
+  static constexpr int kK = 0;
+  static constexpr int kKBytes = kTile * 128 * kElem;
+  static constexpr int kV = kK + kKBytes;
+  static constexpr int kQStage = kBQ * D * kElem;    // one 64-row sub-tile of Q (or dO)
+  static constexpr int kQ = kV + kTile * D * kElem;  // kQStages x Q
   static constexpr int kDO = kQ + kQStages * kQStage;  // kQStages x dO
-  static constexpr int kDSBytes = kTile * kBQ * 2;   // dS^T: 128 keys x 64 queries bf16
-  static constexpr int kDS = kDO + kQStages * kQStage;  // 2 buffers
-  static constexpr int kStats = kDS + 2 * kDSBytes;  // kQStages x (64 lse2 + 64 D_i) fp32
+  static constexpr int kDSBytes = kTile * kBQ * kElem;  // dS^T: 128 keys x 64 queries
+  static constexpr int kDS = kDO + kQStages * kQStage;  // kDSBufs buffers
+  static constexpr int kStats = kDS + kDSBufs * kDSBytes;  // kQStages x (64 lse2 + 64 D_i) fp32
   static constexpr int kList = kStats + kQStages * 2 * kBQ * 4;  // column list, uint16
   static constexpr int kBar = kList + kMaxList * 2;
   enum { KV_FULL, QDO_FULL0, QDO_FULL1, QDO_FULL2, QDO_EMPTY0, QDO_EMPTY1, QDO_EMPTY2, SDP_FULL, DP_FREE,
-         DS_READY, DS_EMPTY0, DS_EMPTY1, DQ_FULL, DQ_EMPTY, ACC_FULL, DRAIN, kNumBars };
+         DS_READY, DS_EMPTY0, DS_EMPTY1, DQ_FULL, DQ_EMPTY, ACC_FULL, DRAIN,
+         QT_GO0, QT_GO1, QT_READY0, QT_READY1, KT_READY,  // fp32 path: operand transposes
+         kNumBars };
   static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort, [2] zero flag
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-template <int D>
+// fp32 path.  kind::tf32 MMAs take K-major operands only, so the products that
+// contract over queries (dV, dK) need Q^T and dO^T, and dQ^T needs K^T.  The
+// dQ-drain warpgroup makes them in shared memory.  Layout of an fp32 operand
+// with 128-byte swizzle: atoms of 32 columns x R rows, element (row, col) at
+// (col / 32) * R * 128 + row * 128 + ((((col % 32) / 4) ^ (row % 8)) * 16) + (col % 4) * 4.
+__device__ __forceinline__ uint32_t f32_sw128_off(int row, int col, int rows) {
+  return (uint32_t)((col >> 5) * rows * 128 + row * 128 + ((((col & 31) >> 2) ^ (row & 7)) << 4) + (col & 3) * 4);
+}
+
+// In-place transpose of a 64 x 64 fp32 tile (Q or dO sub-tile [q][d] -> [d][q]) by 128 threads,
+// rounding to tf32.  Named barrier 1 separates the reads from the writes.
+__device__ __forceinline__ void transpose64_f32(uint8_t* t, int tid) {
+  uint32_t v[32];
+#pragma unroll
+  for (int it = 0; it < 32; ++it) {
+    const int e = it * 128 + tid;
+    v[it] = *reinterpret_cast<const uint32_t*>(t + f32_sw128_off(e >> 6, e & 63, 64));
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+  for (int it = 0; it < 32; ++it) {
+    const int e = it * 128 + tid;
+    *reinterpret_cast<uint32_t*>(t + f32_sw128_off(e & 63, e >> 6, 64)) = round_tf32(__uint_as_float(v[it]));
+  }
+}
+
+// AND of a flag over the 128 drain threads (named barrier 1): every thread reaches it after its own
+// bounded wait, so the threads leave or enter a transpose (which synchronises on barrier 1) together.
+__device__ __forceinline__ bool all_drain_threads(bool v) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((int)v)
+      : "memory");
+  return r != 0;
+}
+
+// K [128 keys][64 d] -> K^T [64 d][128 keys], both fp32 with 128-byte swizzle, by 128 threads.
+__device__ __forceinline__ void transpose_k_f32(const uint8_t* k, uint8_t* kt, int tid) {
+#pragma unroll 8
+  for (int it = 0; it < 64; ++it) {
+    const int e = it * 128 + tid, key = e >> 6, d = e & 63;
+    const float x = *reinterpret_cast<const float*>(k + f32_sw128_off(key, d, kTile));
+    *reinterpret_cast<uint32_t*>(kt + f32_sw128_off(d, key, 64)) = round_tf32(x);
+  }
+}
+
+template <int D, bool F32>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const BwdParams p) {
-  using S = BwdSmem<D>;
+  using S = BwdSmem<D, F32>;
   constexpr int NS = S::kQStages;
+  constexpr int NDS = S::kDSBufs;
+  constexpr int kAtomElems = 128 / S::kElem;  // elements per 128-byte swizzle span
+  constexpr int kAtoms = D * S::kElem / 128;   // swizzle-atom columns of a K / V / Q / dO row
+  constexpr int kKStep = F32 ? 8 : 16;         // elements per UMMA K step (32 bytes)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,14 +163,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(S::DP_FREE), 2 * kTile);
     mbar_init(bar(S::DS_READY), 2 * kTile);
     mbar_init(bar(S::DQ_EMPTY), kTile);
+    mbar_init(bar(S::QT_READY0), kTile);
+    mbar_init(bar(S::QT_READY1), kTile);
+    mbar_init(bar(S::KT_READY), kTile);
     *abort_flag = 0;
     misc[2] = 0;
     fence_barrier_init();
   }
   for (int t = threadIdx.x; t < cnt; t += kBwdThreads) list[t] = (uint16_t)__ldg(entries + t);
-  if (D == 64) {  // K^T as a 128-row MMA operand: rows d >= 64 read this zero block
-    uint4* z = reinterpret_cast<uint4*>(smem + S::kK + kTile * 64 * 2);
-    for (int t = threadIdx.x; t < kTile * 64 * 2 / 16; t += blockDim.x) z[t] = make_uint4(0, 0, 0, 0);
+  if (!F32 && kAtoms * 128 * kTile < S::kKBytes) {  // K^T as a 128-row MMA operand: rows d >= D read zeros
+    uint4* z = reinterpret_cast<uint4*>(smem + S::kK + kAtoms * 128 * kTile);
+    for (int t = threadIdx.x; t < (S::kKBytes - kAtoms * 128 * kTile) / 16; t += blockDim.x)
+      z[t] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (warp == 13) {
@@ -120,8 +185,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  // TMEM columns: S^T / P^T double buffer [0,64) [64,128), dP^T [128,192), dQ^T [192,256), dV, dK
-  const uint32_t tdP = tmem + 128, tdQ = tmem + 192, tdV = tmem + 256, tdK = tmem + 384;
+  // TMEM columns: S^T / P^T double buffer [0,64) [64,128), dP^T [128,192), dQ^T [192,256), dV, dK;
+  // fp32 (D = 64): dS^T [320,384) as the TMEM operand of dK
+  const uint32_t tdP = tmem + 128, tdQ = tmem + 192, tdV = tmem + 256, tdK = tmem + 384, tdS = tmem + 320;
   auto sub_q0 = [&](int i) { return (int)(list[i >> 1] >> 1) * kTile + (i & 1) * kBQ; };
 
   if (warp == 12) {
@@ -131,10 +197,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&tm_do);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(bar(S::KV_FULL), 2 * kTile * D * 2);
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(k_s + c * 16384, &tm_k, bar(S::KV_FULL), c * 64, h, kt * kTile, b);
-        tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * 64, h, kt * kTile, b);
+      mbar_arrive_expect_tx(bar(S::KV_FULL), 2 * kTile * D * S::kElem);
+      for (int c = 0; c < kAtoms; ++c) {
+        tma_load_4d(k_s + c * 16384, &tm_k, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
+        tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
       }
       for (int i = 0; i < nsub; ++i) {
         const int st = i % NS, use = i / NS;
@@ -145,9 +211,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int q0 = sub_q0(i);
         const uint32_t fb = bar(S::QDO_FULL0 + st);
         mbar_arrive_expect_tx(fb, 2 * S::kQStage + 2 * kBQ * 4);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(q_s + st * S::kQStage + c * 8192, &tm_q, fb, c * 64, h, q0, b);
-          tma_load_4d(do_s + st * S::kQStage + c * 8192, &tm_do, fb, c * 64, h, q0, b);
+        for (int c = 0; c < kAtoms; ++c) {
+          tma_load_4d(q_s + st * S::kQStage + c * 8192, &tm_q, fb, c * kAtomElems, h, q0, b);
+          tma_load_4d(do_s + st * S::kQStage + c * 8192, &tm_do, fb, c * kAtomElems, h, q0, b);
         }
         bulk_load(smem_u32(stats + st * 2 * kBQ), p.lse2 + bh * p.n_q + q0, kBQ * 4, fb);
         bulk_load(smem_u32(stats + st * 2 * kBQ + kBQ), p.dvec + bh * p.n_q + q0, kBQ * 4, fb);
@@ -156,9 +222,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 13) {
     // ------------------------------------------------------------- MMA role
     if (lane == 0 && cnt > 0) {
-      constexpr uint32_t kIdSdp = idesc_bf16(128, kBQ, false, false);  // S^T, dP^T: [key][q]
-      constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);     // dV, dK: [key][d], B MN-major
-      constexpr uint32_t kIdDq = idesc_bf16(128, kBQ, true, true);     // dQ^T: [d][q], A and B MN-major
+      // S^T, dP^T: [key][q]; dV, dK: [key][d] with B MN-major; dQ^T: [d][q] with A and B MN-major
+      constexpr uint32_t kIdSdp = F32 ? idesc_tf32(128, kBQ, false, false) : idesc_bf16(128, kBQ, false, false);
+      constexpr uint32_t kIdAcc = F32 ? idesc_tf32(128, D, false, true) : idesc_bf16(128, D, false, true);
+      constexpr uint32_t kIdDq = F32 ? idesc_tf32(128, kBQ, true, true) : idesc_bf16(128, kBQ, true, true);
       // descriptor words (128-byte swizzle, SBO = 8 rows x 128 B); per k-step only the low word moves
       constexpr uint32_t kHi = desc_hi(1024);
       constexpr uint32_t kStageW = S::kQStage >> 4, kDSW = S::kDSBytes >> 4;
@@ -170,28 +237,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto issue_s = [&](int i) {  // S^T_i = K Q_i^T
         const uint32_t qa = lo_q + (i % NS) * kStageW, tS = tmem + (i & 1) * 64;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < D / kKStep; ++k) {
           const uint32_t okv = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, oq = ((k >> 2) * 8192 + (k & 3) * 32) >> 4;
-          umma_ss_w(tS, lo_k + okv, kHi, qa + oq, kHi, kIdSdp, k > 0 ? 1u : 0u);
+          umma_ss_w<F32>(tS, lo_k + okv, kHi, qa + oq, kHi, kIdSdp, k > 0 ? 1u : 0u);
         }
       };
       auto issue_dp = [&](int i) {  // dP^T_i = V dO_i^T
         const uint32_t da = lo_do + (i % NS) * kStageW;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < D / kKStep; ++k) {
           const uint32_t okv = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, oq = ((k >> 2) * 8192 + (k & 3) * 32) >> 4;
-          umma_ss_w(tdP, lo_v + okv, kHi, da + oq, kHi, kIdSdp, k > 0 ? 1u : 0u);
+          umma_ss_w<F32>(tdP, lo_v + okv, kHi, da + oq, kHi, kIdSdp, k > 0 ? 1u : 0u);
         }
       };
+      // fp32: every operand K-major (atoms of 32 columns); Q^T / dO^T replace Q / dO in their stage once
+      // S^T and dP^T have read them, K^T sits after K, dS is stored [q][key]
+      constexpr uint32_t kIdAccT = idesc_tf32(128, D, false, false), kIdDqT = idesc_tf32(128, kBQ, false, false);
+      const uint32_t lo_ktk = desc_lo(k_s + kTile * D * S::kElem, 16);
+      auto toff = [](int k) -> uint32_t { return ((k >> 2) * 8192 + (k & 3) * 32) >> 4; };  // 64-row atoms
       bool ok = mbar_wait(bar(S::KV_FULL), 0, abort_flag) && mbar_wait(bar(S::QDO_FULL0), 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0);
         issue_dp(0);
         umma_commit(bar(S::SDP_FULL));
+        if constexpr (F32) umma_commit(bar(S::QT_GO0));
       }
       for (int i = 0; ok && i < nsub; ++i) {
-        const int st = i % NS, bi = i & 1;
+        const int st = i % NS, bi = i % NDS;
         if (i + 1 < nsub) {  // next sub-tile's S^T (other buffer) and dP^T, overlapping this sub-tile's softmax
           if (!mbar_wait(bar(S::QDO_FULL0 + (i + 1) % NS), ((i + 1) / NS) & 1, abort_flag)) {
             ok = false;
@@ -206,35 +279,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
           issue_dp(i + 1);
           umma_commit(bar(S::SDP_FULL));
+          if constexpr (F32) umma_commit(bar(S::QT_GO0 + (i + 1) % NS));
         }
         if (!mbar_wait(bar(S::DS_READY), i & 1, abort_flag)) {
           ok = false;
           break;
         }
+        if constexpr (F32) {
+          if (!mbar_wait(bar(S::QT_READY0 + st), (i / NS) & 1, abort_flag) ||
+              (i == 0 && !mbar_wait(bar(S::KT_READY), 0, abort_flag))) {
+            ok = false;
+            break;
+          }
+        }
         tc_fence_after();
         const uint32_t qmn = lo_qmn + st * kStageW, domn = lo_domn + st * kStageW;
         const uint32_t dsa = lo_ds + bi * kDSW, dsb = lo_dsmn + bi * kDSW;
-        const uint32_t tP = tmem + bi * 64;
-        // dV += P^T dO (P^T bf16 in TMEM, 16 queries = 8 columns per step; dO MN-major).  Queries
-        // [0, 32) of P^T sit in columns [0, 16) of the buffer, queries [32, 64) in columns [32, 48).
+        const uint32_t tP = tmem + (i & 1) * 64;
+        if constexpr (F32) {
+          // dV += P^T dO^T-operand, dK += dS^T Q^T-operand (A from TMEM, query q in column q)
 #pragma unroll
-        for (int k = 0; k < kBQ / 16; ++k)
-          umma_ts_w(tdV, tP + (k >> 1) * 32 + (k & 1) * 8, domn + ((k * 2048) >> 4), kHi, kIdAcc,
-                    (i > 0 || k > 0) ? 1u : 0u);
-        // dK += dS^T Q (dS^T K-major in smem, one swizzle atom wide; Q MN-major)
+          for (int k = 0; k < kBQ / kKStep; ++k) {
+            const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
+            umma_ts_w<true>(tdV, tP + k * 8, lo_do + st * kStageW + toff(k), kHi, kIdAccT, acc);
+            umma_ts_w<true>(tdK, tdS + k * 8, lo_q + st * kStageW + toff(k), kHi, kIdAccT, acc);
+          }
+          umma_commit(bar(S::QDO_EMPTY0 + st));
+          if (i > 0 && !mbar_wait(bar(S::DQ_EMPTY), (i - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // dQ^T = K^T dS^T: A = K^T (rows d >= 64 read the next atom; those output rows are ignored),
+          // B = dS stored [q][key]
 #pragma unroll
-        for (int k = 0; k < kBQ / 16; ++k)
-          umma_ss_w(tdK, dsa + ((k * 32) >> 4), kHi, qmn + ((k * 2048) >> 4), kHi, kIdAcc, (i > 0 || k > 0) ? 1u : 0u);
-        umma_commit(bar(S::QDO_EMPTY0 + st));
-        if (i > 0 && !mbar_wait(bar(S::DQ_EMPTY), (i - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
+          for (int k = 0; k < kTile / kKStep; ++k)
+            umma_ss_w<true>(tdQ, lo_ktk + toff(k), kHi, lo_ds + toff(k), kHi, kIdDqT, k > 0 ? 1u : 0u);
+        } else {
+          // dV += P^T dO (P^T in TMEM, 8 columns per K step; dO MN-major): queries [0, 32) of P^T are
+          // packed in columns [0, 16) of the buffer, queries [32, 64) in columns [32, 48).
+#pragma unroll
+          for (int k = 0; k < kBQ / kKStep; ++k)
+            umma_ts_w<false>(tdV, tP + (k >> 1) * 32 + (k & 1) * 8, domn + ((k * kKStep * 128) >> 4), kHi, kIdAcc,
+                             (i > 0 || k > 0) ? 1u : 0u);
+          // dK += dS^T Q (dS^T K-major in smem; Q MN-major)
+#pragma unroll
+          for (int k = 0; k < kBQ / kKStep; ++k)
+            umma_ss_w<false>(tdK, dsa + (((k >> 2) * 16384 + (k & 3) * 32) >> 4), kHi,
+                             qmn + ((k * kKStep * 128) >> 4), kHi, kIdAcc, (i > 0 || k > 0) ? 1u : 0u);
+          umma_commit(bar(S::QDO_EMPTY0 + st));
+          if (i > 0 && !mbar_wait(bar(S::DQ_EMPTY), (i - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // dQ^T = K^T dS^T (K^T: M = d, MN-major; dS^T as B: N = q, MN-major; 16 keys per step)
+#pragma unroll
+          for (int k = 0; k < kTile / kKStep; ++k)
+            umma_ss_w<false>(tdQ, lo_kt + ((k * kKStep * 128) >> 4), kHi, dsb + ((k * kKStep * 128) >> 4), kHi,
+                             kIdDq, k > 0 ? 1u : 0u);
         }
-        tc_fence_after();
-        // dQ^T = K^T dS^T (K^T: M = d, MN-major; dS^T as B: N = q, MN-major; 16 keys per step)
-#pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          umma_ss_w(tdQ, lo_kt + ((k * 2048) >> 4), kHi, dsb + ((k * 2048) >> 4), kHi, kIdDq, k > 0 ? 1u : 0u);
         umma_commit(bar(S::DQ_FULL));
         umma_commit(bar(S::DS_EMPTY0 + bi));
       }
@@ -256,14 +360,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int32_t uts = p.vec[2] ? __ldg(p.vec[2] + voff) : 0, ute = p.vec[3] ? __ldg(p.vec[3] + voff) : 0;
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
-      const int st = i % NS, bi = i & 1;
+      const int st = i % NS, bi = i % NDS, sb = i & 1;  // Q/dO stage, dS^T buffer, S^T buffer
       const int q0 = sub_q0(i) + c0;
       const bool partial = list[i >> 1] & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(S::SDP_FULL), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t sd[64];  // [0, 32): S^T row, [32, 64): dP^T row (this warpgroup's queries)
-      tmem_ld32x2(tmem + bi * 64 + c0 + lane_addr, tdP + c0 + lane_addr, sd);
+      tmem_ld32x2(tmem + sb * 64 + c0 + lane_addr, tdP + c0 + lane_addr, sd);
       tc_fence_before();
       mbar_arrive(bar(S::DP_FREE));  // dP^T columns may be overwritten by the next sub-tile
       ok = __all_sync(0xffffffffu, mbar_wait(bar(S::QDO_FULL0 + st), (i / NS) & 1, abort_flag));
@@ -280,7 +384,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
-      uint32_t pk[16], dk[16];
+      uint32_t pk[F32 ? 32 : 16], dk[F32 ? 32 : 16];  // bf16 pairs or tf32-rounded fp32
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
         const float4 L = l2[c4], Dd = dd[c4];
@@ -294,23 +398,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           p0 = ((mbits >> qc) & 1) ? 0.f : p0;
           p1 = ((mbits >> (qc + 1)) & 1) ? 0.f : p1;
           const uint64_t ds2 = mul2(f2pack(p0, p1), add2(((uint64_t)sd[32 + qc + 1] << 32) | sd[32 + qc], nd2));
-          pk[qc >> 1] = pack_bf16(p0, p1);
-          dk[qc >> 1] = pack_bf16(f2lo(ds2), f2hi(ds2));
+          if constexpr (F32) {
+            pk[qc] = round_tf32(p0);
+            pk[qc + 1] = round_tf32(p1);
+            dk[qc] = round_tf32(f2lo(ds2));
+            dk[qc + 1] = round_tf32(f2hi(ds2));
+          } else {
+            pk[qc >> 1] = pack_bf16(p0, p1);
+            dk[qc >> 1] = pack_bf16(f2lo(ds2), f2hi(ds2));
+          }
         }
       }
       // P^T (bf16 pairs) into 16 columns of this warpgroup's own S^T range (already read)
-      tmem_st16(tmem + bi * 64 + c0 + lane_addr, pk);
-      if (i >= 2) {  // dS^T buffer bi free: the dK / dQ^T MMAs of sub-tile i-2 have read it
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DS_EMPTY0 + bi), ((i >> 1) - 1) & 1, abort_flag));
+      if constexpr (F32)
+        tmem_st32(tmem + sb * 64 + c0 + lane_addr, pk);
+      else
+        tmem_st16(tmem + sb * 64 + c0 + lane_addr, pk);
+      if (i >= NDS) {  // dS^T buffer bi free: the dK / dQ^T MMAs of sub-tile i-NDS have read it
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DS_EMPTY0 + bi), ((i / NDS) - 1) & 1, abort_flag));
         if (!ok) break;
       }
-      // dS^T row r, queries [c0, c0+32): four 16-byte chunks, 128-byte swizzle (chunk c at c ^ (r & 7))
-      uint8_t* ds_row = smem + S::kDS + bi * S::kDSBytes + r * 128;
+      if constexpr (F32) {
+        // dS^T into TMEM (the A operand of dK), and dS [q][key] K-major (the B operand of dQ^T):
+        // for one query the warp's 32 keys fill one 128-byte row of atom r / 32
+        tmem_st32(tdS + c0 + lane_addr, dk);
+        uint8_t* ds_col = smem + S::kDS + (r >> 5) * 8192 + (r & 3) * 4;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int chunk = 4 * hf + c;
-        *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
-            make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+        for (int qc = 0; qc < 32; ++qc) {
+          const int q = c0 + qc;
+          *reinterpret_cast<uint32_t*>(ds_col + q * 128 + ((((r & 31) >> 2) ^ (q & 7)) << 4)) = dk[qc];
+        }
+      } else {
+        // dS^T row r, queries [c0, c0+32), 128-byte swizzle (16-byte chunk c of a row at c ^ (r & 7)):
+        // four chunks of the row's single atom
+
+        uint8_t* ds_row = smem + S::kDS + bi * S::kDSBytes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = 4 * hf + c;
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -319,12 +447,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (!ok) record_failure(p.status, abort_flag, 13);
   } else {
     // ------------------------------------- dQ drain role (row = d), warps 8-11
+    // fp32: also the operand transposes (K^T once; Q^T and dO^T per sub-tile, in place after S^T and
+    // dP^T have read the stage)
     const int d = threadIdx.x - 256;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q * D;
     bool ok = true;
-    for (int i = 0; i < nsub; ++i) {
+    if constexpr (F32) {
+      if (nsub > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::KV_FULL), 0, abort_flag));
+        if (ok) {
+          transpose_k_f32(smem + S::kK, smem + S::kK + kTile * D * S::kElem, d);
+          fence_proxy_async_smem();
+          mbar_arrive(bar(S::KT_READY));
+        }
+      }
+    }
+    for (int i = 0; ok && i < nsub; ++i) {
       const int q0 = sub_q0(i);
+      if constexpr (F32) {
+        const int st = i % NS;
+        ok = all_drain_threads(mbar_wait(bar(S::QT_GO0 + st), (i / NS) & 1, abort_flag));
+        if (!ok) break;
+        transpose64_f32(smem + S::kQ + st * S::kQStage, d);
+        transpose64_f32(smem + S::kDO + st * S::kQStage, d);
+        fence_proxy_async_smem();
+        mbar_arrive(bar(S::QT_READY0 + st));
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DQ_FULL), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -354,7 +503,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
     }
     const float mul = is_dk ? p.scale : 1.f;
-    __nv_bfloat16* out = (is_dk ? p.dk : p.dv) + (((int64_t)b * p.n_k + (int64_t)kt * kTile + r) * p.H + h) * D;
+    const int64_t orow = (((int64_t)b * p.n_k + (int64_t)kt * kTile + r) * p.H + h) * D;
     const uint32_t tsrc = (is_dk ? tdK : tdV) + lane_addr;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -365,13 +514,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) a[c] = 0u;
       }
-      uint32_t pk[16];
+      if constexpr (F32) {
+        float* dst = static_cast<float*>(is_dk ? p.dk : p.dv) + orow + cc * 32;
 #pragma unroll
-      for (int c = 0; c < 32; c += 2)
-        pk[c >> 1] = pack_bf16(__uint_as_float(a[c]) * mul, __uint_as_float(a[c + 1]) * mul);
+        for (int v4 = 0; v4 < 8; ++v4)
+          st_global_v4(dst + v4 * 4, __float_as_uint(__uint_as_float(a[4 * v4]) * mul),
+                       __float_as_uint(__uint_as_float(a[4 * v4 + 1]) * mul),
+                       __float_as_uint(__uint_as_float(a[4 * v4 + 2]) * mul),
+                       __float_as_uint(__uint_as_float(a[4 * v4 + 3]) * mul));
+      } else {
+        uint32_t pk[16];
 #pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4)
-        st_global_v4(out + cc * 32 + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        for (int c = 0; c < 32; c += 2)
+          pk[c >> 1] = pack_bf16(__uint_as_float(a[c]) * mul, __uint_as_float(a[c + 1]) * mul);
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(is_dk ? p.dk : p.dv) + orow + cc * 32;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          st_global_v4(dst + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
     }
   }
 
@@ -385,9 +545,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // D_i = dO_i . O_i, log2-domain LSE (+inf for empty rows so that P = 0), and
 // a cleared dQ accumulator.  One thread per (b, i, h) row.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
-                                                       const __nv_bfloat16* __restrict__ dout,
+template <int D, bool F32>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ o, const void* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ dvec, float* __restrict__ acc, int B,
                                                        int H, int n_q) {
@@ -397,19 +556,29 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
     const int h = (int)(t % H);
     const int64_t bi = t / H;
     const int i = (int)(bi % n_q), b = (int)(bi / n_q);
-    const uint4* po = reinterpret_cast<const uint4*>(o + t * D);
-    const uint4* pd = reinterpret_cast<const uint4*>(dout + t * D);
     float s = 0.f;
+    if constexpr (F32) {
+      const float4* po = reinterpret_cast<const float4*>(static_cast<const float*>(o) + t * D);
+      const float4* pd = reinterpret_cast<const float4*>(static_cast<const float*>(dout) + t * D);
 #pragma unroll 4
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 a = __ldg(po + c), g = __ldg(pd + c);
-      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+      for (int c = 0; c < D / 4; ++c) {
+        const float4 a = __ldg(po + c), g = __ldg(pd + c);
+        s = fmaf(a.x, g.x, fmaf(a.y, g.y, fmaf(a.z, g.z, fmaf(a.w, g.w, s))));
+      }
+    } else {
+      const uint4* po = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + t * D);
+      const uint4* pd = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dout) + t * D);
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 a = __ldg(po + c), g = __ldg(pd + c);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[u]));
-        const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[u]));
-        s = fmaf(fa.x, fg.x, s);
-        s = fmaf(fa.y, fg.y, s);
+        for (int u = 0; u < 4; ++u) {
+          const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[u]));
+          const float2 fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[u]));
+          s = fmaf(fa.x, fg.x, s);
+          s = fmaf(fa.y, fg.y, s);
+        }
       }
     }
     const int64_t out = ((int64_t)b * H + h) * n_q + i;
@@ -426,8 +595,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 // dQ[b, i, h, :] = scale * acc for one 64-row block per CTA: the block (a
 // contiguous 16 x D x 4 fp32 run) is read coalesced into shared memory (padded
 // against bank conflicts), then each thread writes 8 consecutive d of one row.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+template <int D, bool F32>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, void* __restrict__ dq,
                                                      int B, int H, int n_q, float scale) {
   __shared__ float4 buf[16 * D + 2 * D];  // one float4 of padding per 8
   const int blocks_per_bh = n_q / 64;
@@ -447,8 +616,16 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
       const float4 f = buf[k + (k >> 3)];
       x[c] = (u == 0 ? f.x : u == 1 ? f.y : u == 2 ? f.z : f.w) * scale;
     }
-    __nv_bfloat16* row = dq + (((int64_t)b * n_q + (int64_t)qb * 64 + q) * H + h) * D + d0;
-    st_global_v4(row, pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    const int64_t off = (((int64_t)b * n_q + (int64_t)qb * 64 + q) * H + h) * D + d0;
+    if constexpr (F32) {
+      float* row = static_cast<float*>(dq) + off;
+      st_global_v4(row, __float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+      st_global_v4(row + 4, __float_as_uint(x[4]), __float_as_uint(x[5]), __float_as_uint(x[6]),
+                   __float_as_uint(x[7]));
+    } else {
+      __nv_bfloat16* row = static_cast<__nv_bfloat16*>(dq) + off;
+      st_global_v4(row, pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    }
   }
 }
 
@@ -468,10 +645,10 @@ BwdLayout bwd_layout(const fm_attn_args* a) {
   return L;
 }
 
-template <int D>
+template <int D, bool F32>
 fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], const void* o,
                      const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws, cudaStream_t stream) {
-  using S = BwdSmem<D>;
+  using S = BwdSmem<D, F32>;
   static_assert(S::kAlloc <= 227 * 1024, "backward shared memory exceeds the per-CTA limit");
   const BwdLayout L = bwd_layout(a);
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -479,14 +656,12 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   float* lse2 = reinterpret_cast<float*>(w + L.lse2);
   float* dvec = reinterpret_cast<float*>(w + L.dvec);
   CUtensorMap tq, tdo, tk, tv;
-  if (!encode_tmap_bf16_4d(&tq, a->q, D, a->H, a->n_q, a->B, kBQ) ||
-      !encode_tmap_bf16_4d(&tdo, dout, D, a->H, a->n_q, a->B, kBQ) ||
-      !encode_tmap_bf16_4d(&tk, a->k, D, a->H, a->n_k, a->B, kTile) ||
-      !encode_tmap_bf16_4d(&tv, a->v, D, a->H, a->n_k, a->B, kTile))
+  auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
+  if (!enc(&tq, a->q, D, a->H, a->n_q, a->B, kBQ) || !enc(&tdo, dout, D, a->H, a->n_q, a->B, kBQ) ||
+      !enc(&tk, a->k, D, a->H, a->n_k, a->B, kTile) || !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile))
     return FM_ERR_CUDA;
   const int64_t rows = (int64_t)a->B * a->n_q * a->H;
-  bwd_prep_kernel<D><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec, acc, a->B,
+  bwd_prep_kernel<D, F32><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(o, dout, lse, lse2, dvec, acc, a->B,
       a->H, a->n_q);
   BwdParams p;
   p.col_count = meta->col_count;
@@ -495,8 +670,8 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.lse2 = lse2;
   p.dvec = dvec;
   p.dq_acc = acc;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dk = dk;
+  p.dv = dv;
   p.status = device_status_ptr();
   p.B = a->B;
   p.H = a->H;
@@ -507,11 +682,12 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.T_k = a->n_k / kTile;
   p.scale = a->scale;
   p.scale_log2 = a->scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) != cudaSuccess)
+  if (cudaFuncSetAttribute(bwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
+      cudaSuccess)
     return FM_ERR_CUDA;
-  bwd_kernel<D><<<dim3(p.T_k, p.H, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, p);
-  bwd_dq_kernel<D><<<(unsigned)((int64_t)a->B * a->H * (a->n_q / 64)), 256, 0, stream>>>(
-      acc, static_cast<__nv_bfloat16*>(dq), a->B, a->H, a->n_q, a->scale);
+  bwd_kernel<D, F32><<<dim3(p.T_k, p.H, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, p);
+  bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (a->n_q / 64)), 256, 0, stream>>>(
+      acc, dq, a->B, a->H, a->n_q, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 
@@ -538,8 +714,9 @@ fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) || ws_bytes < fm_attn_bwd_workspace_bytes(a))
     return FM_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return a->D == 64 ? fm::launch_bwd<64>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s)
-                    : fm::launch_bwd<128>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s);
+  if (a->dtype == 1) return fm::launch_bwd<64, true>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s);
+  return a->D == 64 ? fm::launch_bwd<64, false>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s)
+                    : fm::launch_bwd<128, false>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s);
 }
 
 }  // extern "C"

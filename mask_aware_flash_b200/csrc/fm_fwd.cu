@@ -43,16 +43,18 @@ struct FwdParams {
   const int32_t* row_count;    // [B, Hm, T_q]
   const int32_t* row_entries;  // [B, Hm, T_q, T_k]
   const int32_t* vec[4];       // [B, Hm, n_k] or null
-  __nv_bfloat16* o;            // [B, n_q, H, D]
+  const float* v32;            // fp32 V [B, n_k, H, D] (fp32 path: loaded transposed by the load warp)
+  void* o;                     // [B, n_q, H, D], bf16 or fp32
   float* lse;                  // [B, H, n_q]
   int* status;
   int B, H, Hm, n_q, n_k, T_q, T_k, n_pairs;
   float scale_log2;            // softmax scale * log2(e), > 0
 };
 
-template <int D>
+template <int D, bool F32>
 struct FwdSmem {
-  static constexpr int kTileBytes = kTile * D * 2;  // 128 rows x D bf16 (D/64 swizzle-atom columns)
+  static constexpr int kElem = F32 ? 4 : 2;
+  static constexpr int kTileBytes = kTile * D * kElem;  // 128 rows x D elements (128-byte swizzle-atom columns)
   static constexpr int kQ = 0;                      // Q0, Q1
   static constexpr int kK = kQ + 2 * kTileBytes;    // K ring, 2 slots
   static constexpr int kV = kK + 2 * kTileBytes;    // V ring, 2 slots
@@ -88,11 +90,36 @@ struct MergedList {
   }
 };
 
+// fp32 path: kind::tf32 MMAs read both operands K-major, so PV needs V^T
+// ([d][key], keys contiguous).  One warp copies a 128-key fp32 V tile from
+// global memory into that layout (128-byte swizzle; four atoms of 32 keys,
+// D rows of 128 bytes each), rounding to tf32 on the way: element (d, key) sits
+// at (key / 32) * D * 128 + d * 128 + ((((key % 32) / 4) ^ (d % 8)) * 16) + (key % 4) * 4.
 template <int D>
+__device__ __forceinline__ void load_vt_f32(uint8_t* dst, const float* src, int64_t row_stride, int lane) {
+  constexpr int kQuads = D / 4;
+#pragma unroll 4
+  for (int e = lane; e < kTile * kQuads; e += 32) {
+    const int key = e / kQuads, dq = e % kQuads;
+    const float4 x = __ldg(reinterpret_cast<const float4*>(src + key * row_stride) + dq);
+    const float xs[4] = {x.x, x.y, x.z, x.w};
+    uint8_t* col = dst + (key >> 5) * (D * 128) + (key & 3) * 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int d = 4 * dq + j;
+      *reinterpret_cast<uint32_t*>(col + d * 128 + ((((key & 31) >> 2) ^ (d & 7)) << 4)) = round_tf32(xs[j]);
+    }
+  }
+}
+
+template <int D, bool F32>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using S = FwdSmem<D>;
+  using S = FwdSmem<D, F32>;
+  constexpr int kAtomElems = 128 / S::kElem;        // elements per 128-byte swizzle span
+  constexpr int kAtoms = D * S::kElem / 128;         // swizzle-atom columns per tile row
+  constexpr int kKStep = F32 ? 8 : 16;               // elements per UMMA K step (32 bytes)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,58 +170,85 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ load role
-    if (lane == 0 && any) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
+    // bf16: lane 0 issues every TMA load.  fp32: the whole warp walks the list
+    // (V^T is copied by all 32 lanes), lane 0 still issuing the TMA loads.
+    if ((F32 || lane == 0) && any) {
+      auto wait_all = [&](uint32_t bb, uint32_t ph) {
+        bool r = mbar_wait(bb, ph, abort_flag);
+        if constexpr (F32) r = __all_sync(0xffffffffu, r);
+        return r;
+      };
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        mbar_arrive_expect_tx(bar(S::Q_FULL), (has1 ? 2 : 1) * S::kTileBytes);
+        for (int c = 0; c < kAtoms; ++c) {
+          tma_load_4d(q_s + c * 16384, &tm_q, bar(S::Q_FULL), c * kAtomElems, h, qt0 * kTile, b);
+          if (has1)
+            tma_load_4d(q_s + S::kTileBytes + c * 16384, &tm_q, bar(S::Q_FULL), c * kAtomElems, h, qt1 * kTile, b);
+        }
+      }
       int nvec = 0;
       for (int c = 0; c < 4; ++c) nvec += p.vec[c] ? 1 : 0;
-      mbar_arrive_expect_tx(bar(S::Q_FULL), (has1 ? 2 : 1) * S::kTileBytes);
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(q_s + c * 16384, &tm_q, bar(S::Q_FULL), c * 64, h, qt0 * kTile, b);
-        if (has1) tma_load_4d(q_s + S::kTileBytes + c * 16384, &tm_q, bar(S::Q_FULL), c * 64, h, qt1 * kTile, b);
-      }
       MergedList it{list0, list1, n0, n1, 0, 0};
       int kt, c0, c1, e = 0, mcount = 0;
       bool ok = true;
       while (it.next(kt, c0, c1)) {
         const int slot = e & 1;
-        if (e >= 2 && !mbar_wait(bar(S::K_EMPTY0 + slot), ((e >> 1) - 1) & 1, abort_flag)) {
+        if (e >= 2 && !wait_all(bar(S::K_EMPTY0 + slot), ((e >> 1) - 1) & 1)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(S::K_FULL0 + slot), S::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(k_s + slot * S::kTileBytes + c * 16384, &tm_k, bar(S::K_FULL0 + slot), c * 64, h, kt * kTile, b);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(S::K_FULL0 + slot), S::kTileBytes);
+          for (int c = 0; c < kAtoms; ++c)
+            tma_load_4d(k_s + slot * S::kTileBytes + c * 16384, &tm_k, bar(S::K_FULL0 + slot), c * kAtomElems, h,
+                        kt * kTile, b);
+        }
         if (c0 == 1 || c1 == 1) {
           const int mb = mcount & 1;
-          if (mcount >= 2 && !mbar_wait(bar(S::M_EMPTY0 + mb), ((mcount >> 1) - 1) & 1, abort_flag)) {
+          if (mcount >= 2 && !wait_all(bar(S::M_EMPTY0 + mb), ((mcount >> 1) - 1) & 1)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(S::M_FULL0 + mb), 512u * nvec);
-          for (int c = 0; c < 4; ++c)
-            if (p.vec[c])
-              bulk_load(smem_u32(mask_smem + (mb * 4 + c) * kTile), p.vec[c] + bhm * p.n_k + (int64_t)kt * kTile,
-                        512u, bar(S::M_FULL0 + mb));
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar(S::M_FULL0 + mb), 512u * nvec);
+            for (int c = 0; c < 4; ++c)
+              if (p.vec[c])
+                bulk_load(smem_u32(mask_smem + (mb * 4 + c) * kTile), p.vec[c] + bhm * p.n_k + (int64_t)kt * kTile,
+                          512u, bar(S::M_FULL0 + mb));
+          }
           ++mcount;
         }
-        if (e >= 2 && !mbar_wait(bar(S::V_EMPTY0 + slot), ((e >> 1) - 1) & 1, abort_flag)) {
+        if (e >= 2 && !wait_all(bar(S::V_EMPTY0 + slot), ((e >> 1) - 1) & 1)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(S::V_FULL0 + slot), S::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(v_s + slot * S::kTileBytes + c * 16384, &tm_v, bar(S::V_FULL0 + slot), c * 64, h, kt * kTile, b);
+        if constexpr (F32) {
+          load_vt_f32<D>(smem + S::kV + slot * S::kTileBytes,
+                         p.v32 + (((int64_t)b * p.n_k + (int64_t)kt * kTile) * p.H + h) * D, (int64_t)p.H * D, lane);
+          fence_proxy_async_smem();  // generic-proxy stores, read next by the tensor core
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(S::V_FULL0 + slot));
+        } else {
+          mbar_arrive_expect_tx(bar(S::V_FULL0 + slot), S::kTileBytes);
+          for (int c = 0; c < kAtoms; ++c)
+            tma_load_4d(v_s + slot * S::kTileBytes + c * 16384, &tm_v, bar(S::V_FULL0 + slot), c * kAtomElems, h,
+                        kt * kTile, b);
+        }
         ++e;
       }
-      if (!ok) record_failure(p.status, abort_flag, 1);
+      if (!ok && lane == 0) record_failure(p.status, abort_flag, 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA role
     if (lane == 0 && any) {
-      constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false, false);  // S[q][kv]: Q K-major, K K-major
-      constexpr uint32_t kIdescPV = idesc_bf16(128, D, false, true);     // O[q][d]:  P (TMEM), V MN-major
+      // S[q][kv]: Q K-major, K K-major; O[q][d]: P from TMEM, V MN-major (bf16) or V^T K-major (tf32,
+      // which takes K-major operands only)
+      constexpr uint32_t kIdescQK = F32 ? idesc_tf32(128, 128, false, false) : idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdescPV = F32 ? idesc_tf32(128, D, false, false) : idesc_bf16(128, D, false, true);
+      constexpr int kPvSteps = kTile / kKStep;  // UMMA K steps over the 128 kv rows
       MergedList it{list0, list1, n0, n1, 0, 0};
       int kt, c0, c1, kn, n0c, n1c;
       bool ok = mbar_wait(bar(S::Q_FULL), 0, abort_flag);
@@ -203,14 +257,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool acc[2] = {false, false};
       // descriptor words: 128-byte swizzle, SBO = 8 rows x 128 B; per k-step only the low word moves
       constexpr uint32_t kHi = desc_hi(1024);
-      const uint32_t lo_q = desc_lo(q_s, 16), lo_k = desc_lo(k_s, 16), lo_v = desc_lo(v_s, 16384);
+      const uint32_t lo_q = desc_lo(q_s, 16), lo_k = desc_lo(k_s, 16), lo_v = desc_lo(v_s, F32 ? 16 : 16384);
+      // k-th PV step (kKStep kv rows): bf16 V rows of 128 B; tf32 V^T atoms of 32 keys x D rows
+      auto pv_off = [&](int k) -> uint32_t {
+        return F32 ? (((k >> 2) * (D * 128) + (k & 3) * 32) >> 4) : ((k * kKStep * 128) >> 4);
+      };
       constexpr uint32_t kTileW = S::kTileBytes >> 4;  // one tile, in 16-byte descriptor units
       auto issue_s = [&](int t, int kslot) {  // S_t = Q_t K^T
         const uint32_t qa = lo_q + t * kTileW, ka = lo_k + kslot * kTileW;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;  // swizzle-atom column, 16-element K step
-          umma_ss_w(tmem + t * 256, qa + off, kHi, ka + off, kHi, kIdescQK, k > 0 ? 1u : 0u);
+        for (int k = 0; k < D / kKStep; ++k) {
+          const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;  // swizzle-atom column, 32-byte K step
+          umma_ss_w<F32>(tmem + t * 256, qa + off, kHi, ka + off, kHi, kIdescQK, k > 0 ? 1u : 0u);
         }
         umma_commit(bar(S::S_FULL0 + t));
       };
@@ -245,8 +303,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tc_fence_after();
             const uint32_t va = lo_v + slot * kTileW;
 #pragma unroll
-            for (int k = 0; k < kTile / 32; ++k)  // 16 kv rows per step; P columns advance 8 (bf16 pairs)
-              umma_ts_w(tO, tS + k * 8, va + ((k * 2048) >> 4), kHi, kIdescPV, (acc[t] || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kPvSteps / 2; ++k)  // kKStep kv rows per step; P columns advance 8 per step
+              umma_ts_w<F32>(tO, tS + k * 8, va + pv_off(k), kHi, kIdescPV, (acc[t] || k > 0) ? 1u : 0u);
             if (!mbar_wait(bar(S::P_FULL0 + t), np[t] & 1, abort_flag)) {
               ok = false;
               break;
@@ -254,8 +312,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             ++np[t];
             tc_fence_after();
 #pragma unroll
-            for (int k = kTile / 32; k < kTile / 16; ++k)
-              umma_ts_w(tO, tS + k * 8, va + ((k * 2048) >> 4), kHi, kIdescPV, 1u);
+            for (int k = kPvSteps / 2; k < kPvSteps; ++k)
+              umma_ts_w<F32>(tO, tS + k * 8, va + pv_off(k), kHi, kIdescPV, 1u);
             umma_commit(bar(S::O_DONE0 + t));
             acc[t] = true;
           }
@@ -341,7 +399,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float rq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[32];
+          // bf16: 32 packed pairs per half; fp32: 64 tf32-rounded values per half
+          uint32_t pk[F32 ? 64 : 32];
 #pragma unroll
           for (int c = 0; c < kTile / 2; c += 2) {
             const int cs = hh * (kTile / 2) + c;
@@ -357,9 +416,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             const int k = (c >> 1) & 3;
             rs2[k] = add2(rs2[k], f2pack(p0, p1));
-            const uint32_t w = pack_bf16(p0, p1);
-            rq[k] = add_bf16x2_to_f32(w, rq[k]);
-            pk[c >> 1] = w;
+            if constexpr (F32) {
+              const uint32_t w0 = round_tf32(p0), w1 = round_tf32(p1);
+              rq[k] += __uint_as_float(w0) + __uint_as_float(w1);
+              pk[c] = w0;
+              pk[c + 1] = w1;
+            } else {
+              const uint32_t w = pack_bf16(p0, p1);
+              rq[k] = add_bf16x2_to_f32(w, rq[k]);
+              pk[c >> 1] = w;
+            }
           }
           if (hh == 0 && __any_sync(0xffffffffu, move && j > 0)) {
             // O holds the sum over earlier tiles: wait for the last PV, rescale it in TMEM
@@ -376,7 +442,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tmem_st16(tO + cc * 16, orr);
             }
           }
-          tmem_st32(tS + hh * 32, pk);
+          if constexpr (F32)
+            tmem_st64(tS + hh * 64, pk);
+          else
+            tmem_st32(tS + hh * 32, pk);
           tc_fence_before();
           mbar_arrive(bar((hh ? S::P_FULL0 : S::P_HALF0) + t));
         }
@@ -401,7 +470,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (!ok) record_failure(p.status, abort_flag, 5);
     // epilogue: O = O / l, LSE = (m + log2 l) ln 2; empty rows: O = 0, LSE = -inf
     if (live_tile) {
-      __nv_bfloat16* orow = p.o + (((int64_t)b * p.n_q + i) * p.H + h) * D;
+      const int64_t orow = (((int64_t)b * p.n_q + i) * p.H + h) * D;
       const bool live = ok && j > 0 && l_run > kLiveSum;
       bool have_o = false;
       if (ok && j > 0) {
@@ -419,13 +488,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) orr[c] = 0u;
         }
-        uint32_t pk[16];
+        if constexpr (F32) {
+          float* dst = static_cast<float*>(p.o) + orow + cc * 32;
 #pragma unroll
-        for (int c = 0; c < 32; c += 2)
-          pk[c >> 1] = pack_bf16(__uint_as_float(orr[c]) * inv, __uint_as_float(orr[c + 1]) * inv);
+          for (int v4 = 0; v4 < 8; ++v4)
+            st_global_v4(dst + v4 * 4, __float_as_uint(__uint_as_float(orr[4 * v4]) * inv),
+                         __float_as_uint(__uint_as_float(orr[4 * v4 + 1]) * inv),
+                         __float_as_uint(__uint_as_float(orr[4 * v4 + 2]) * inv),
+                         __float_as_uint(__uint_as_float(orr[4 * v4 + 3]) * inv));
+        } else {
+          uint32_t pk[16];
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          st_global_v4(orow + cc * 32 + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          for (int c = 0; c < 32; c += 2)
+            pk[c >> 1] = pack_bf16(__uint_as_float(orr[c]) * inv, __uint_as_float(orr[c + 1]) * inv);
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) + orow + cc * 32;
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(dst + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
       }
       p.lse[((int64_t)b * p.H + h) * p.n_q + i] = live ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
     }
@@ -439,21 +519,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool F32>
 fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], void* o,
                      float* lse, cudaStream_t stream) {
-  using S = FwdSmem<D>;
+  using S = FwdSmem<D, F32>;
   static_assert(S::kAlloc <= 227 * 1024, "forward shared memory exceeds the per-CTA limit");
   CUtensorMap tq, tk, tv;
-  if (!encode_tmap_bf16_4d(&tq, a->q, D, a->H, a->n_q, a->B, kTile) ||
-      !encode_tmap_bf16_4d(&tk, a->k, D, a->H, a->n_k, a->B, kTile) ||
-      !encode_tmap_bf16_4d(&tv, a->v, D, a->H, a->n_k, a->B, kTile))
+  auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
+  if (!enc(&tq, a->q, D, a->H, a->n_q, a->B, kTile) || !enc(&tk, a->k, D, a->H, a->n_k, a->B, kTile) ||
+      !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile))
     return FM_ERR_CUDA;
   FwdParams p;
   p.row_count = meta->row_count;
   p.row_entries = meta->row_entries;
   for (int c = 0; c < 4; ++c) p.vec[c] = vec ? vec[c] : nullptr;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.v32 = F32 ? static_cast<const float*>(a->v) : nullptr;
+  p.o = o;
   p.lse = lse;
   p.status = device_status_ptr();
   p.B = a->B;
@@ -465,9 +546,10 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.T_k = a->n_k / kTile;
   p.n_pairs = (p.T_q + 1) / 2;
   p.scale_log2 = a->scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) != cudaSuccess)
+  if (cudaFuncSetAttribute(fwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
+      cudaSuccess)
     return FM_ERR_CUDA;
-  fwd_kernel<D><<<dim3(p.n_pairs, p.H, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, p);
+  fwd_kernel<D, F32><<<dim3(p.n_pairs, p.H, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 
@@ -478,8 +560,9 @@ fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const
   if (!a || !meta) return FM_ERR_INVALID_ARG;
   if (a->B < 1 || a->H < 1 || a->n_q < 1 || a->n_k < 1 || a->B > 65535 || a->H > 65535) return FM_ERR_INVALID_ARG;
   if (!(a->scale > 0.f) || a->scale > 3.0e38f) return FM_ERR_INVALID_ARG;  // positive and finite
-  if (a->dtype != 0) return FM_ERR_UNSUPPORTED;
+  if (a->dtype != 0 && a->dtype != 1) return FM_ERR_UNSUPPORTED;
   if (a->D != 64 && a->D != 128) return FM_ERR_UNSUPPORTED;
+  if (a->dtype == 1 && a->D != 64) return FM_ERR_UNSUPPORTED;  // fp32 tiles of D=128 exceed shared memory
   if (a->n_q % kTile || a->n_k % kTile) return FM_ERR_UNSUPPORTED;
   if (a->n_k / kTile > kMaxList || a->n_q / kTile > kMaxList) return FM_ERR_UNSUPPORTED;  // lists held in smem
   if (!a->q || !a->k || !a->v) return FM_ERR_INVALID_ARG;
@@ -505,5 +588,7 @@ extern "C" fm_status fm_attn_fwd(const fm_attn_args* a, const fm_mask_meta* meta
   if (!o || !lse || (reinterpret_cast<uintptr_t>(o) & 15) || (reinterpret_cast<uintptr_t>(lse) & 3))
     return FM_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return a->D == 64 ? fm::launch_fwd<64>(a, meta, vec, o, lse, s) : fm::launch_fwd<128>(a, meta, vec, o, lse, s);
+  if (a->dtype == 1) return fm::launch_fwd<64, true>(a, meta, vec, o, lse, s);
+  return a->D == 64 ? fm::launch_fwd<64, false>(a, meta, vec, o, lse, s)
+                    : fm::launch_fwd<128, false>(a, meta, vec, o, lse, s);
 }

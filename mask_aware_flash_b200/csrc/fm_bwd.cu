@@ -375,14 +375,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float4* l2 = reinterpret_cast<const float4*>(stats + st * 2 * kBQ + c0);
       const float4* dd = reinterpret_cast<const float4*>(stats + st * 2 * kBQ + kBQ + c0);
       // row-interval test (partial tiles only) as a mask of this key's masked queries
-      uint32_t mbits = 0;
-      if (partial) {
-#pragma unroll
-        for (int qc = 0; qc < 32; ++qc) {
-          const int64_t q = q0 + qc;
-          mbits |= (((lts <= q && q < lte) || (uts <= q && q < ute)) ? 1u : 0u) << qc;
-        }
-      }
+      const uint32_t mbits = partial ? (interval_bits32(lts, lte, q0) | interval_bits32(uts, ute, q0)) : 0u;
       const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
       uint32_t pk[F32 ? 32 : 16], dk[F32 ? 32 : 16];  // bf16 pairs or tf32-rounded fp32
 #pragma unroll

@@ -405,6 +405,33 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {  // three-in
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
+// Bits of the 32 rows base .. base+31 that lie in the half-open interval [start, end)
+// (bit r = row base + r).  start and end are any int32 values: they are clamped to
+// [base, base + 32] before any subtraction, so nothing overflows.
+__device__ __forceinline__ uint32_t interval_bits32(int32_t start, int32_t end, int32_t base) {
+  const int a = min(max(start, base), base + 32) - base, b = min(max(end, base), base + 32) - base;
+  return b > a ? ((0xFFFFFFFFu >> (32 - b)) & (0xFFFFFFFFu << a)) : 0u;
+}
+
+// Transpose of four 32 x 32 bit matrices held one row per lane: on return bit l of
+// lane r's word w[j] is bit r of lane l's word w[j] on entry.  Five butterfly
+// stages; at stage s, lanes l and l ^ s swap the off-diagonal s x s blocks.
+__device__ __forceinline__ void bit_transpose32x4(uint32_t (&w)[4], int lane) {
+  constexpr uint32_t kLow[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int st = 0; st < 5; ++st) {
+    const int s = 16 >> st;
+    const bool upper = (lane & s) != 0;
+    const uint32_t keep = upper ? ~kLow[st] : kLow[st];  // bits this lane keeps
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, w[j], s);
+      const uint32_t t = upper ? (y >> s) : (y << s);
+      w[j] = (w[j] & keep) | (t & ~keep);
+    }
+  }
+}
+
 // the two bf16 halves of a packed pair, as fp32 (exact)
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

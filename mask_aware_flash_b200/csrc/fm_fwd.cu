@@ -366,13 +366,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // row-interval test (partial tiles only): masked scores -> -inf
           ok = __all_sync(0xffffffffu, mbar_wait(bar(S::M_FULL0 + mb), (mcount >> 1) & 1, abort_flag));
           if (!ok) break;
+          // Lane l turns key columns l, l+32, l+64, l+96 into words of "masked rows of this warp";
+          // a bit transpose then gives each row's thread one bit per column.  32-column blocks
+          // with no masked entry in the warp are skipped.
           const int32_t* mv = mask_smem + mb * 4 * kTile;
+          const int32_t w0 = qt * kTile + (warp & 3) * 32;  // this warp's first row
+          uint32_t mw[4];
 #pragma unroll
-          for (int c = 0; c < kTile; ++c) {
+          for (int jb = 0; jb < 4; ++jb) {
+            const int c = jb * 32 + lane;
             const int32_t lts = has[0] ? mv[c] : p.n_q, lte = has[1] ? mv[kTile + c] : p.n_q;
             const int32_t uts = has[2] ? mv[2 * kTile + c] : 0, ute = has[3] ? mv[3 * kTile + c] : 0;
-            const bool msk = (lts <= i && i < lte) || (uts <= i && i < ute);
-            s[c] = msk ? __float_as_uint(kNegInf) : s[c];
+            mw[jb] = interval_bits32(lts, lte, w0) | interval_bits32(uts, ute, w0);
+          }
+          bit_transpose32x4(mw, lane);
+#pragma unroll
+          for (int jb = 0; jb < 4; ++jb) {
+            if (__any_sync(0xffffffffu, mw[jb] != 0u)) {
+#pragma unroll
+              for (int l = 0; l < 32; ++l)
+                s[jb * 32 + l] = ((mw[jb] >> l) & 1u) ? __float_as_uint(kNegInf) : s[jb * 32 + l];
+            }
           }
         }
         // row maximum: four independent three-input max chains

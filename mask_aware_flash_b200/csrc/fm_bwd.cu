@@ -130,6 +130,7 @@ template <int D, bool F32>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                const BwdParams p) {
   using S = BwdSmem<D, F32>;
   constexpr int NS = S::kQStages;
@@ -169,6 +170,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     *abort_flag = 0;
     misc[2] = 0;
     fence_barrier_init();
+    if (cnt > 0) {  // K and V first: their latency overlaps the list copy and the TMEM allocation
+      fence_proxy_async_smem();
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(bar(S::KV_FULL), 2 * kTile * D * S::kElem);
+      for (int c = 0; c < kAtoms; ++c) {
+        tma_load_4d(k_s + c * 16384, &tm_k, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
+        tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
+      }
+    }
   }
   for (int t = threadIdx.x; t < cnt; t += kBwdThreads) list[t] = (uint16_t)__ldg(entries + t);
   if (!F32 && kAtoms * 128 * kTile < S::kKBytes) {  // K^T as a 128-row MMA operand: rows d >= D read zeros
@@ -193,15 +204,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 12) {
     // ------------------------------------------------------------ load role
     if (lane == 0 && cnt > 0) {
-      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_q);  // (K and V were issued at the start)
       prefetch_tmap(&tm_do);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(bar(S::KV_FULL), 2 * kTile * D * S::kElem);
-      for (int c = 0; c < kAtoms; ++c) {
-        tma_load_4d(k_s + c * 16384, &tm_k, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
-        tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
-      }
       for (int i = 0; i < nsub; ++i) {
         const int st = i % NS, use = i / NS;
         if (use >= 1 && !mbar_wait(bar(S::QDO_EMPTY0 + st), (use - 1) & 1, abort_flag)) {
@@ -486,6 +490,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 
   // ---------------------------------------------- epilogue: dV (warps 0-3), dK (warps 4-7)
+  // Each warpgroup stages its 128 x D tile (output dtype, 128-byte swizzle) in the Q (dV) or dO (dK)
+  // stage buffers, which no load or MMA touches any more, and one of its threads TMA-stores it.
   if (warp < 8) {
     const int r = threadIdx.x & 127;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
@@ -496,8 +502,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
     }
     const float mul = is_dk ? p.scale : 1.f;
-    const int64_t orow = (((int64_t)b * p.n_k + (int64_t)kt * kTile + r) * p.H + h) * D;
     const uint32_t tsrc = (is_dk ? tdK : tdV) + lane_addr;
+    uint8_t* stage = smem + (is_dk ? S::kDO : S::kQ);
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t a[32];
@@ -507,24 +513,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) a[c] = 0u;
       }
-      if constexpr (F32) {
-        float* dst = static_cast<float*>(is_dk ? p.dk : p.dv) + orow + cc * 32;
+      if constexpr (F32) {  // 32 fp32 = one atom row: chunks 0..7 of atom cc
+        uint8_t* row = stage + cc * 16384 + r * 128;
 #pragma unroll
-        for (int v4 = 0; v4 < 8; ++v4)
-          st_global_v4(dst + v4 * 4, __float_as_uint(__uint_as_float(a[4 * v4]) * mul),
-                       __float_as_uint(__uint_as_float(a[4 * v4 + 1]) * mul),
-                       __float_as_uint(__uint_as_float(a[4 * v4 + 2]) * mul),
-                       __float_as_uint(__uint_as_float(a[4 * v4 + 3]) * mul));
-      } else {
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) =
+              make_uint4(__float_as_uint(__uint_as_float(a[4 * ch]) * mul),
+                         __float_as_uint(__uint_as_float(a[4 * ch + 1]) * mul),
+                         __float_as_uint(__uint_as_float(a[4 * ch + 2]) * mul),
+                         __float_as_uint(__uint_as_float(a[4 * ch + 3]) * mul));
+      } else {  // 32 bf16 = half an atom row: chunks 4 (cc & 1) .. +3 of atom cc / 2
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2)
           pk[c >> 1] = pack_bf16(__uint_as_float(a[c]) * mul, __uint_as_float(a[c + 1]) * mul);
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(is_dk ? p.dk : p.dv) + orow + cc * 32;
+        uint8_t* row = stage + (cc >> 1) * 16384 + r * 128;
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          st_global_v4(dst + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        for (int ch = 0; ch < 4; ++ch)
+          *reinterpret_cast<uint4*>(row + ((((cc & 1) * 4 + ch) ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
       }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(is_dk ? 3 : 2, 128);
+    if (r == 0) {
+      for (int c = 0; c < kAtoms; ++c)
+        tma_store_4d(is_dk ? &tm_dk : &tm_dv, smem_u32(stage + c * 16384), c * kAtomElems, h, kt * kTile, b);
+      bulk_commit_group();
+      bulk_wait_group_read0();
     }
   }
 
@@ -648,10 +664,11 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   float* acc = reinterpret_cast<float*>(w + L.acc);
   float* lse2 = reinterpret_cast<float*>(w + L.lse2);
   float* dvec = reinterpret_cast<float*>(w + L.dvec);
-  CUtensorMap tq, tdo, tk, tv;
+  CUtensorMap tq, tdo, tk, tv, tdk, tdv;
   auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
   if (!enc(&tq, a->q, D, a->H, a->n_q, a->B, kBQ) || !enc(&tdo, dout, D, a->H, a->n_q, a->B, kBQ) ||
-      !enc(&tk, a->k, D, a->H, a->n_k, a->B, kTile) || !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile))
+      !enc(&tk, a->k, D, a->H, a->n_k, a->B, kTile) || !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile) ||
+      !enc(&tdk, dk, D, a->H, a->n_k, a->B, kTile) || !enc(&tdv, dv, D, a->H, a->n_k, a->B, kTile))
     return FM_ERR_CUDA;
   const int64_t rows = (int64_t)a->B * a->n_q * a->H;
   bwd_prep_kernel<D, F32><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(o, dout, lse, lse2, dvec, acc, a->B,
@@ -678,7 +695,7 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   if (cudaFuncSetAttribute(bwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
       cudaSuccess)
     return FM_ERR_CUDA;
-  bwd_kernel<D, F32><<<dim3(p.T_k, p.H, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, p);
+  bwd_kernel<D, F32><<<dim3(p.T_k, p.H, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
   bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (a->n_q / 64)), 256, 0, stream>>>(
       acc, dq, a->B, a->H, a->n_q, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;

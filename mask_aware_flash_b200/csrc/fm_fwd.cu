@@ -115,7 +115,8 @@ __device__ __forceinline__ void load_vt_f32(uint8_t* dst, const float* src, int6
 template <int D, bool F32>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const FwdParams p) {
   using S = FwdSmem<D, F32>;
   constexpr int kAtomElems = 128 / S::kElem;        // elements per 128-byte swizzle span
   constexpr int kAtoms = D * S::kElem / 128;         // swizzle-atom columns per tile row
@@ -154,6 +155,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     *abort_flag = 0;
     misc[2] = 0;  // a flag nothing raises: lets the final drain wait ignore aborts
     fence_barrier_init();
+    if (n0 + n1 > 0) {  // Q first: its latency overlaps the list copy and the TMEM allocation
+      fence_proxy_async_smem();
+      prefetch_tmap(&tm_q);
+      mbar_arrive_expect_tx(bar(S::Q_FULL), (has1 ? 2 : 1) * S::kTileBytes);
+      for (int c = 0; c < kAtoms; ++c) {
+        tma_load_4d(q_s + c * 16384, &tm_q, bar(S::Q_FULL), c * kAtomElems, h, qt0 * kTile, b);
+        if (has1)
+          tma_load_4d(q_s + S::kTileBytes + c * 16384, &tm_q, bar(S::Q_FULL), c * kAtomElems, h, qt1 * kTile, b);
+      }
+    }
   }
   // both row lists into shared memory (coalesced)
   for (int t = threadIdx.x; t < n0; t += kFwdThreads) list0[t] = (uint16_t)__ldg(rows0 + t);
@@ -178,16 +189,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if constexpr (F32) r = __all_sync(0xffffffffu, r);
         return r;
       };
-      if (lane == 0) {
-        prefetch_tmap(&tm_q);
+      if (lane == 0) {  // (Q was issued at the start)
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_arrive_expect_tx(bar(S::Q_FULL), (has1 ? 2 : 1) * S::kTileBytes);
-        for (int c = 0; c < kAtoms; ++c) {
-          tma_load_4d(q_s + c * 16384, &tm_q, bar(S::Q_FULL), c * kAtomElems, h, qt0 * kTile, b);
-          if (has1)
-            tma_load_4d(q_s + S::kTileBytes + c * 16384, &tm_q, bar(S::Q_FULL), c * kAtomElems, h, qt1 * kTile, b);
-        }
       }
       int nvec = 0;
       for (int c = 0; c < 4; ++c) nvec += p.vec[c] ? 1 : 0;
@@ -484,7 +488,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (!ok) record_failure(p.status, abort_flag, 5);
     // epilogue: O = O / l, LSE = (m + log2 l) ln 2; empty rows: O = 0, LSE = -inf
     if (live_tile) {
-      const int64_t orow = (((int64_t)b * p.n_q + i) * p.H + h) * D;
       const bool live = ok && j > 0 && l_run > kLiveSum;
       bool have_o = false;
       if (ok && j > 0) {
@@ -493,6 +496,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
       }
       const float inv = live ? 1.f / lq_run : 0.f;
+      // O tile staged in this tile's Q buffer (every S_t product has finished once O_DONE_t has
+      // fired; the PV product does not read Q), 128-byte swizzle, then TMA-stored by one thread
+      uint8_t* stage = smem + S::kQ + t * S::kTileBytes;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t orr[32];
@@ -502,24 +508,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) orr[c] = 0u;
         }
-        if constexpr (F32) {
-          float* dst = static_cast<float*>(p.o) + orow + cc * 32;
+        if constexpr (F32) {  // 32 fp32 = one atom row
+          uint8_t* row = stage + cc * 16384 + r * 128;
 #pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            st_global_v4(dst + v4 * 4, __float_as_uint(__uint_as_float(orr[4 * v4]) * inv),
-                         __float_as_uint(__uint_as_float(orr[4 * v4 + 1]) * inv),
-                         __float_as_uint(__uint_as_float(orr[4 * v4 + 2]) * inv),
-                         __float_as_uint(__uint_as_float(orr[4 * v4 + 3]) * inv));
-        } else {
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) =
+                make_uint4(__float_as_uint(__uint_as_float(orr[4 * ch]) * inv),
+                           __float_as_uint(__uint_as_float(orr[4 * ch + 1]) * inv),
+                           __float_as_uint(__uint_as_float(orr[4 * ch + 2]) * inv),
+                           __float_as_uint(__uint_as_float(orr[4 * ch + 3]) * inv));
+        } else {  // 32 bf16 = half an atom row
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2)
             pk[c >> 1] = pack_bf16(__uint_as_float(orr[c]) * inv, __uint_as_float(orr[c + 1]) * inv);
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) + orow + cc * 32;
+          uint8_t* row = stage + (cc >> 1) * 16384 + r * 128;
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_global_v4(dst + v4 * 8, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          for (int ch = 0; ch < 4; ++ch)
+            *reinterpret_cast<uint4*>(row + ((((cc & 1) * 4 + ch) ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(2 + t, 128);
+      if (r == 0) {
+        for (int c = 0; c < kAtoms; ++c)
+          tma_store_4d(&tm_o, smem_u32(stage + c * 16384), c * kAtomElems, h, qt * kTile, b);
+        bulk_commit_group();
+        bulk_wait_group_read0();
       }
       p.lse[((int64_t)b * p.H + h) * p.n_q + i] = live ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
     }
@@ -538,10 +554,10 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
                      float* lse, cudaStream_t stream) {
   using S = FwdSmem<D, F32>;
   static_assert(S::kAlloc <= 227 * 1024, "forward shared memory exceeds the per-CTA limit");
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
   if (!enc(&tq, a->q, D, a->H, a->n_q, a->B, kTile) || !enc(&tk, a->k, D, a->H, a->n_k, a->B, kTile) ||
-      !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile))
+      !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile) || !enc(&to, o, D, a->H, a->n_q, a->B, kTile))
     return FM_ERR_CUDA;
   FwdParams p;
   p.row_count = meta->row_count;
@@ -563,7 +579,7 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   if (cudaFuncSetAttribute(fwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
       cudaSuccess)
     return FM_ERR_CUDA;
-  fwd_kernel<D, F32><<<dim3(p.n_pairs, p.H, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, p);
+  fwd_kernel<D, F32><<<dim3(p.n_pairs, p.H, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

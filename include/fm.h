@@ -75,6 +75,14 @@ typedef struct {
  *                                (kt << 1) | is_partial, kt ascending
  *   col_count   [B, Hm, T_k], col_entries [B, Hm, T_k, T_q]: the transpose,
  *                                (qt << 1) | is_partial, qt ascending
+ *   fwd_order   [B, Hm, ceil(T_q/2)] int32: query-tile pairs (2p, 2p+1) by descending
+ *                                row_count[2p] + row_count[2p+1], ties by ascending p
+ *   bwd_order   [B, Hm, T_k] int32: key tiles by descending col_count, ties by
+ *                                ascending index
+ *   (both the identity order when T_q or T_k exceeds 4096).  The attention kernels
+ *   dispatch the CTAs of each (b, h) in these orders, longest first, one (b, h)
+ *   after the other (a scheduling aid with no counterpart in the paper; results
+ *   do not depend on it).
  * Rule (per query tile rows [r0, r1), key tile min/max as above):
  *   skip    = (maxLTS <= r0 && minLTE >= r1) || (maxUTS <= r0 && minUTE >= r1)
  *   full    = !skip && (minLTS >= r1 || maxLTE <= r0) && (minUTS >= r1 || maxUTE <= r0)
@@ -89,6 +97,8 @@ typedef struct {
   int32_t* col_count;
   int32_t* col_entries;
   uint8_t* tile_class;
+  int32_t* fwd_order;
+  int32_t* bwd_order;
 } fm_mask_meta;
 
 /* Bytes of workspace fm_build_mask_meta needs for `d` (0 if d is invalid). */

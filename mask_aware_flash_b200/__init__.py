@@ -41,7 +41,8 @@ class MaskDesc(ctypes.Structure):
 class MaskMetaC(ctypes.Structure):
     _fields_ = [("d", MaskDesc), ("tile_minmax", ctypes.c_void_p), ("row_count", ctypes.c_void_p),
                 ("row_entries", ctypes.c_void_p), ("col_count", ctypes.c_void_p),
-                ("col_entries", ctypes.c_void_p), ("tile_class", ctypes.c_void_p)]
+                ("col_entries", ctypes.c_void_p), ("tile_class", ctypes.c_void_p),
+                ("fwd_order", ctypes.c_void_p), ("bwd_order", ctypes.c_void_p)]
 
 
 class AttnArgs(ctypes.Structure):
@@ -130,6 +131,8 @@ class MaskMeta:
         self.col_count = view(c.col_count, torch.int32, (B, Hm, self.T_k))
         self.col_entries = view(c.col_entries, torch.int32, (B, Hm, self.T_k, self.T_q))
         self.tile_class = view(c.tile_class, torch.uint8, (B, Hm, self.T_q, self.T_k))
+        self.fwd_order = view(c.fwd_order, torch.int32, (B, Hm, (self.T_q + 1) // 2))
+        self.bwd_order = view(c.bwd_order, torch.int32, (B, Hm, self.T_k))
 
 
 def fm_mask_meta_workspace_bytes(B, Hm, n_q, n_k) -> int:

@@ -38,6 +38,7 @@ constexpr float kPosInf = __builtin_huge_valf();
 struct BwdParams {
   const int32_t* col_count;    // [B, Hm, T_k]
   const int32_t* col_entries;  // [B, Hm, T_k, T_q]
+  const int32_t* order;        // [B, Hm, T_k] dispatch order (longest first)
   const int32_t* vec[4];       // [B, Hm, n_k] or null
   const float* lse2;           // [B, H, n_q] log2-domain LSE, +inf on empty rows
   const float* dvec;           // [B, H, n_q] D_i = dO_i . O_i
@@ -46,6 +47,7 @@ struct BwdParams {
   void* dv;
   int* status;
   int B, H, Hm, n_q, n_k, T_q, T_k;
+  int group;                   // heads dispatched together
   float scale, scale_log2;
 };
 
@@ -141,9 +143,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (group * T_k, ceil(H / group), B): a group of heads at a time, rank by rank over the
+  // group's heads (rank r takes the key tile with the r-th longest column list); the group is sized
+  // so that its heads' Q, dO and dQ accumulator stay in L2
+  const int h = (int)blockIdx.y * p.group + (int)(blockIdx.x % p.group), b = blockIdx.z;
+  if (h >= p.H) return;  // partial last group
   const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
+  const int kt = __ldg(p.order + bhm * p.T_k + blockIdx.x / p.group);
   const int64_t bh = (int64_t)b * p.H + h;
   const int cnt = __ldg(p.col_count + bhm * p.T_k + kt);
   const int nsub = 2 * cnt;  // two 64-row sub-tiles per listed 128-row query tile
@@ -676,6 +682,7 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   BwdParams p;
   p.col_count = meta->col_count;
   p.col_entries = meta->col_entries;
+  p.order = meta->bwd_order;
   for (int c = 0; c < 4; ++c) p.vec[c] = vec ? vec[c] : nullptr;
   p.lse2 = lse2;
   p.dvec = dvec;
@@ -690,12 +697,13 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.n_k = a->n_k;
   p.T_q = a->n_q / kTile;
   p.T_k = a->n_k / kTile;
+  p.group = dispatch_group(p.H, (double)a->n_q * D * (2 * S::kElem + 4));  // Q, dO, fp32 dQ accumulator
   p.scale = a->scale;
   p.scale_log2 = a->scale * 1.4426950408889634f;
   if (cudaFuncSetAttribute(bwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
       cudaSuccess)
     return FM_ERR_CUDA;
-  bwd_kernel<D, F32><<<dim3(p.T_k, p.H, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
+  bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
   bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (a->n_q / 64)), 256, 0, stream>>>(
       acc, dq, a->B, a->H, a->n_q, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;

@@ -483,6 +483,13 @@ __device__ __forceinline__ int ld_nc_i32(const int32_t* p) {
 // ---------------------------------------------------------------------------
 namespace fm {
 int* device_status_ptr();  // per-device status word; nullptr on failure
+// Heads whose CTAs an attention kernel dispatches together: as many as keep the
+// per-head bytes that all CTAs of a head re-read within 32 MiB of L2 (at least 1,
+// at most H).
+inline int dispatch_group(int H, double bytes_per_head) {
+  int g = (int)((32.0 * 1024 * 1024) / (bytes_per_head > 1.0 ? bytes_per_head : 1.0));
+  return g < 1 ? 1 : (g > H ? H : g);
+}
 bool encode_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t n, uint64_t B,
                          uint32_t box_rows);
 bool encode_tmap_f32_4d(CUtensorMap* map, const void* base, uint64_t D, uint64_t H, uint64_t n, uint64_t B,

@@ -42,12 +42,14 @@ constexpr float kLiveSum = 1e-20f;  // a live row's sum is >= ~1; masked scores 
 struct FwdParams {
   const int32_t* row_count;    // [B, Hm, T_q]
   const int32_t* row_entries;  // [B, Hm, T_q, T_k]
+  const int32_t* order;        // [B, Hm, n_pairs] dispatch order (longest first)
   const int32_t* vec[4];       // [B, Hm, n_k] or null
   const float* v32;            // fp32 V [B, n_k, H, D] (fp32 path: loaded transposed by the load warp)
   void* o;                     // [B, n_q, H, D], bf16 or fp32
   float* lse;                  // [B, H, n_q]
   int* status;
   int B, H, Hm, n_q, n_k, T_q, T_k, n_pairs;
+  int group;                   // heads dispatched together
   float scale_log2;            // softmax scale * log2(e), > 0
 };
 
@@ -124,11 +126,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = p.n_pairs - 1 - (int)blockIdx.x;  // long (late causal) query tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // grid (group * n_pairs, ceil(H / group), B): the CTAs of a group of heads are dispatched together,
+  // rank by rank over the group's heads (rank r takes the pair with the r-th longest list, so the
+  // longest start first); the group is sized so that its heads' K/V stay in L2
+  const int h = (int)blockIdx.y * p.group + (int)(blockIdx.x % p.group), b = blockIdx.z;
+  if (h >= p.H) return;  // partial last group
+  const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
+  const int pair = __ldg(p.order + bhm * p.n_pairs + blockIdx.x / p.group);
   const int qt0 = 2 * pair, qt1 = 2 * pair + 1;
   const bool has1 = qt1 < p.T_q;
-  const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
   const int32_t* rows0 = p.row_entries + (bhm * p.T_q + qt0) * p.T_k;
   const int32_t* rows1 = rows0 + p.T_k;
   const int n0 = __ldg(p.row_count + bhm * p.T_q + qt0);
@@ -562,6 +568,7 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   FwdParams p;
   p.row_count = meta->row_count;
   p.row_entries = meta->row_entries;
+  p.order = meta->fwd_order;
   for (int c = 0; c < 4; ++c) p.vec[c] = vec ? vec[c] : nullptr;
   p.v32 = F32 ? static_cast<const float*>(a->v) : nullptr;
   p.o = o;
@@ -575,11 +582,12 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.T_q = a->n_q / kTile;
   p.T_k = a->n_k / kTile;
   p.n_pairs = (p.T_q + 1) / 2;
+  p.group = dispatch_group(p.H, 2.0 * a->n_k * D * S::kElem);
   p.scale_log2 = a->scale * 1.4426950408889634f;
   if (cudaFuncSetAttribute(fwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
       cudaSuccess)
     return FM_ERR_CUDA;
-  fwd_kernel<D, F32><<<dim3(p.n_pairs, p.H, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, to, p);
+  fwd_kernel<D, F32><<<dim3(p.group * p.n_pairs, (p.H + p.group - 1) / p.group, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 
@@ -602,7 +610,9 @@ fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const
   if (d.B != a->B || d.n_q != a->n_q || d.n_k != a->n_k || d.tile_q != kTile || d.tile_k != kTile)
     return FM_ERR_INVALID_ARG;
   if (d.Hm != 1 && d.Hm != a->H) return FM_ERR_INVALID_ARG;
-  if (!meta->row_count || !meta->row_entries || !meta->col_count || !meta->col_entries) return FM_ERR_INVALID_ARG;
+  if (!meta->row_count || !meta->row_entries || !meta->col_count || !meta->col_entries || !meta->fwd_order ||
+      !meta->bwd_order)
+    return FM_ERR_INVALID_ARG;
   if (vec)
     for (int c = 0; c < 4; ++c)
       if (reinterpret_cast<uintptr_t>(vec[c]) & 15) return FM_ERR_INVALID_ARG;

@@ -23,6 +23,8 @@ struct MetaParams {
   int32_t* row_entries;   // [BHm, T_q, T_k]
   int32_t* col_count;     // [BHm, T_k]
   int32_t* col_entries;   // [BHm, T_k, T_q]
+  int32_t* fwd_order;     // [BHm, ceil(T_q / 2)]
+  int32_t* bwd_order;     // [BHm, T_k]
   int32_t BHm, n_q, n_k, T_q, T_k;
 };
 
@@ -132,8 +134,57 @@ __global__ void __launch_bounds__(256) meta_lists_kernel(const MetaParams p) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Dispatch orders for the attention kernels (longest first).  One CTA per
+// (b, hm) and direction: blockIdx.y = 0 orders query-tile pairs by the sum of
+// their two row counts, 1 orders key tiles by column count; ties keep
+// ascending index.  Bitonic sort in shared memory of the keys
+// (cost << 16) | (0xFFFF - index), descending; with at most 4096 items and
+// costs below 2^16 the keys are distinct, so the order is deterministic.
+constexpr int kOrderMax = 4096;
+__global__ void __launch_bounds__(1024) meta_order_kernel(const MetaParams p) {
+  __shared__ uint32_t key[kOrderMax];
+  const int bhm = blockIdx.x;
+  const bool fwd = blockIdx.y == 0;
+  const int n = fwd ? (p.T_q + 1) / 2 : p.T_k;
+  int32_t* out = fwd ? p.fwd_order + (int64_t)bhm * n : p.bwd_order + (int64_t)bhm * n;
+  if (p.T_q > kOrderMax || p.T_k > kOrderMax) {  // sizes the attention kernels do not take
+    for (int i = threadIdx.x; i < n; i += blockDim.x) out[i] = i;
+    return;
+  }
+  int np2 = 1;
+  while (np2 < n) np2 <<= 1;
+  const int32_t* rc = p.row_count + (int64_t)bhm * p.T_q;
+  const int32_t* cc = p.col_count + (int64_t)bhm * p.T_k;
+  for (int i = threadIdx.x; i < np2; i += blockDim.x) {
+    uint32_t k = 0;  // padding sorts last
+    if (i < n) {
+      const uint32_t cost = fwd ? (uint32_t)(rc[2 * i] + (2 * i + 1 < p.T_q ? rc[2 * i + 1] : 0)) : (uint32_t)cc[i];
+      k = (cost << 16) | (0xFFFFu - (uint32_t)i);
+    }
+    key[i] = k;
+  }
+  __syncthreads();
+  for (int len = 2; len <= np2; len <<= 1) {
+    for (int j = len >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < np2; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint32_t a = key[i], b = key[ixj];
+          const bool desc = (i & len) == 0;  // descending runs merge into one descending sequence
+          if (desc ? (a < b) : (a > b)) {
+            key[i] = b;
+            key[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) out[i] = (int32_t)(0xFFFFu - (key[i] & 0xFFFFu));
+}
+
 struct MetaLayout {
-  size_t minmax, row_count, row_entries, col_count, col_entries, cls, total;
+  size_t minmax, row_count, row_entries, col_count, col_entries, cls, fwd_order, bwd_order, total;
 };
 
 bool meta_layout(const fm_mask_desc* d, MetaLayout* L) {
@@ -155,6 +206,10 @@ bool meta_layout(const fm_mask_desc* d, MetaLayout* L) {
   off = align256(off + BHm * T_k * T_q * 4);
   L->cls = off;
   off = align256(off + BHm * T_q * T_k);
+  L->fwd_order = off;
+  off = align256(off + BHm * ((T_q + 1) / 2) * 4);
+  L->bwd_order = off;
+  off = align256(off + BHm * T_k * 4);
   L->total = off;
   return true;
 }
@@ -183,6 +238,8 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
   out->col_count = reinterpret_cast<int32_t*>(w + L.col_count);
   out->col_entries = reinterpret_cast<int32_t*>(w + L.col_entries);
   out->tile_class = w + L.cls;
+  out->fwd_order = reinterpret_cast<int32_t*>(w + L.fwd_order);
+  out->bwd_order = reinterpret_cast<int32_t*>(w + L.bwd_order);
 
   fm::MetaParams p;
   p.vec[0] = lts;
@@ -195,6 +252,8 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
   p.row_entries = out->row_entries;
   p.col_count = out->col_count;
   p.col_entries = out->col_entries;
+  p.fwd_order = out->fwd_order;
+  p.bwd_order = out->bwd_order;
   p.BHm = d->B * d->Hm;
   p.n_q = d->n_q;
   p.n_k = d->n_k;
@@ -205,6 +264,7 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
   fm::meta_minmax_kernel<<<(unsigned)((warps_mm + 7) / 8), 256, 0, s>>>(p);
   const int64_t warps_l = (int64_t)p.BHm * (p.T_q > p.T_k ? p.T_q : p.T_k);
   fm::meta_lists_kernel<<<dim3((unsigned)((warps_l + 7) / 8), 2), 256, 0, s>>>(p);
+  fm::meta_order_kernel<<<dim3((unsigned)p.BHm, 2), 1024, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

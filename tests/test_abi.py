@@ -47,7 +47,8 @@ def test_meta_workspace_bytes(L):
     d = fm.MaskDesc(2, 1, 1024, 2048, 128, 128)
     n = L.fm_mask_meta_workspace_bytes(ctypes.byref(d))
     T_q, T_k = 8, 16
-    assert n >= 2 * (T_k * 8 * 4 + T_q * 4 + T_q * T_k * 4 + T_k * 4 + T_k * T_q * 4 + T_q * T_k)
+    assert n >= 2 * (T_k * 8 * 4 + T_q * 4 + T_q * T_k * 4 + T_k * 4 + T_k * T_q * 4 + T_q * T_k + (T_q // 2) * 4
+                     + T_k * 4)
     assert n % 256 == 0
     bad = fm.MaskDesc(2, 1, 1024, 2048, 64, 128)
     assert L.fm_mask_meta_workspace_bytes(ctypes.byref(bad)) == 0
@@ -95,7 +96,7 @@ def _attn(L, n_q=256, n_k=256, D=128, dtype=0, meta_nq=None, Hm=1, H=2):
     m = fm.MaskMetaC()
     m.d = fm.MaskDesc(1, Hm, meta_nq or n_q, n_k, 128, 128)
     m.row_count = m.row_entries = m.col_count = m.col_entries = m.tile_minmax = 0x40000
-    m.tile_class = 0x40000
+    m.tile_class = m.fwd_order = m.bwd_order = 0x40000
     return a, m
 
 
@@ -117,6 +118,9 @@ def test_fwd_rejects_before_launch(L):
         fm.FM_ERR_INVALID_ARG  # misaligned output
     vec_bad = fm.VecArray(0x70004, None, None, None)
     assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec_bad, o, lse, None) == fm.FM_ERR_INVALID_ARG
+    a, m = _attn(L)
+    m.fwd_order = None  # metadata without its dispatch orders
+    assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, o, lse, None) == fm.FM_ERR_INVALID_ARG
 
 
 def test_bwd_rejects_before_launch(L):

@@ -81,6 +81,11 @@ def _check_meta(fm, vt, n_q, n_k):
             ce = meta.col_entries[b, hm].cpu().numpy()
             for kt in range(len(cc)):
                 np.testing.assert_array_equal(ce[kt, :cc[kt]], ref["col_entries"][kt, :cc[kt]])
+            # dispatch orders: longest first, ties by ascending index (stable sort on -cost)
+            rcp = np.concatenate([ref["row_count"], [0]])[: 2 * ((len(rc) + 1) // 2)].reshape(-1, 2).sum(1)
+            np.testing.assert_array_equal(meta.fwd_order[b, hm].cpu().numpy(), np.argsort(-rcp, kind="stable"))
+            np.testing.assert_array_equal(meta.bwd_order[b, hm].cpu().numpy(),
+                                          np.argsort(-ref["col_count"], kind="stable"))
     return meta
 
 

@@ -75,7 +75,7 @@ def test_noalloc_rejects_oversize(fm):
     m = fm.MaskMetaC()
     m.d = fm.MaskDesc(1, 1, n, n, 128, 128)
     m.row_count = m.row_entries = m.col_count = m.col_entries = m.tile_minmax = 0x40000
-    m.tile_class = 0x40000
+    m.tile_class = m.fwd_order = m.bwd_order = 0x40000
     p = [ctypes.c_void_p(0x100000 * (t + 1)) for t in range(6)]
     rc = fm.lib().fm_attn_bwd_noalloc(ctypes.byref(a), ctypes.byref(m), fm.VecArray(None, None, None, None), *p,
                                       None)

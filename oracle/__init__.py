@@ -44,6 +44,7 @@ def _load():
         L.orc_count_unmasked_dense.restype = i64
         L.orc_count_unmasked_intervals.argtypes = [i32, i32, vp, vp, vp, vp]
         L.orc_count_unmasked_intervals.restype = i64
+        L.orc_kv_chunk_pairs.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
         L.orc_tile_meta.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.orc_localize_clip_shift_max.argtypes = [i64, vp, i32, vp, vp, vp]
         L.orc_localize_count.argtypes = [i64, vp, i32, vp, vp, vp]
@@ -86,6 +87,16 @@ def count_unmasked(n_q, n_k, lts, lte, uts, ute) -> int:
     """Unmasked pairs from interval lengths (O(n_k)); equals the dense count."""
     v = [_i32(x) for x in (lts, lte, uts, ute)]
     return int(_load().orc_count_unmasked_intervals(n_q, n_k, *[_ptr(x) for x in v]))
+
+
+def kv_chunk_pairs(n_q, n_k, chunk_len, lts, lte, uts, ute) -> np.ndarray:
+    """[explainer] across-ranks paragraph ("skips key-value chunks that are fully
+    masked"): unmasked (row, key) pairs of rows [0, n_q) per chunk of chunk_len
+    keys; a zero entry is a chunk no row attends to."""
+    v = [None if x is None else _i32(x) for x in (lts, lte, uts, ute)]
+    out = np.empty(-(-n_k // chunk_len), np.int64)
+    _load().orc_kv_chunk_pairs(n_q, n_k, chunk_len, *[None if x is None else _ptr(x) for x in v], out.ctypes.data)
+    return out
 
 
 def tile_meta(n_q, n_k, lts, lte, uts, ute, tile_q=128, tile_k=128) -> dict:

@@ -94,6 +94,19 @@ int64_t orc_count_unmasked_intervals(int32_t n_q, int32_t n_k, const int32_t* lt
   return c;
 }
 
+// Unmasked (row, key) pairs per key chunk of chunk_len keys ([explainer] across-ranks
+// paragraph: the all-gather skips key-value chunks that are fully masked; a chunk with
+// zero pairs is one of them).  Plain: the per-column count above over each chunk's keys.
+void orc_kv_chunk_pairs(int32_t n_q, int32_t n_k, int32_t chunk_len, const int32_t* lts, const int32_t* lte,
+                        const int32_t* uts, const int32_t* ute, int64_t* out) {
+  const int32_t n_chunks = (n_k + chunk_len - 1) / chunk_len;
+  for (int32_t c = 0; c < n_chunks; ++c) {
+    const int32_t j0 = c * chunk_len, j1 = std::min(j0 + chunk_len, n_k);
+    out[c] = orc_count_unmasked_intervals(n_q, j1 - j0, lts ? lts + j0 : nullptr, lte ? lte + j0 : nullptr,
+                                          uts ? uts + j0 : nullptr, ute ? ute + j0 : nullptr);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Tile classification and block lists ([explainer] "sort every tile of the
 // score matrix as fully masked, partly masked or unmasked, using the maximum

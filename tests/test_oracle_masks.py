@@ -260,3 +260,58 @@ def test_dual_chunk_tile_classes_match_global():
         lm = oracle.tile_meta(2 * chunk, N, *loc)
         grows = np.concatenate([np.arange(s // 128, (s + chunk) // 128) for s in starts])
         np.testing.assert_array_equal(lm["cls"], gm["cls"][grows])
+
+
+# ---- KV-chunk pruning counts ------------------------------------------------
+def test_kv_chunk_pairs_dense_brute_force():
+    """Per-chunk unmasked pairs equal the dense mask's count over each chunk's keys
+    (random vectors with out-of-range and empty stretches, ragged last chunk)."""
+    r = np.random.default_rng(21)
+    for _ in range(120):
+        n_q, n_k = int(r.integers(1, 90)), int(r.integers(1, 120))
+        vecs = [r.integers(-5, n_q + 5, n_k).astype(np.int32) for _ in range(4)]
+        cl = int(r.integers(1, n_k + 3))
+        got = oracle.kv_chunk_pairs(n_q, n_k, cl, *vecs)
+        unm = ~oracle.dense_mask(n_q, n_k, *vecs)
+        want = np.add.reduceat(unm.sum(0), np.arange(0, n_k, cl)).astype(np.int64)
+        np.testing.assert_array_equal(got, want)
+
+
+def test_kv_chunk_pairs_null_and_causal_closed_form():
+    N, cl = 1000, 128
+    full = oracle.kv_chunk_pairs(N, N, cl, None, None, None, None)
+    np.testing.assert_array_equal(full, [N * min(cl, N - c * cl) for c in range(-(-N // cl))])
+    spec = synth.mask_causal(N)  # key j is seen by rows j .. N-1
+    got = oracle.kv_chunk_pairs(N, N, cl, *spec.vectors())
+    want = [sum(N - j for j in range(c * cl, min((c + 1) * cl, N))) for c in range(-(-N // cl))]
+    np.testing.assert_array_equal(got, want)
+
+
+def test_kv_chunk_pairs_ranks_partition_global():
+    """Ranks whose chunks partition the query rows: by Theorem 1 their local pairs
+    per KV chunk add up to the global mask's, and a chunk is pruned for a rank
+    exactly when the rank's rows of the global dense mask are all masked there."""
+    r = np.random.default_rng(22)
+    N, nch, cl = 512, 8, 64
+    chunk = N // nch
+    pruned = 0
+    for family in ("causal_document", "share_question", "sliding_window_2k", "prefix_lm_document", "random_eviction"):
+        spec = synth.make_family(family, N, 23)
+        vecs = spec.vectors()
+        glob = oracle.kv_chunk_pairs(N, N, cl, *vecs)
+        dense = oracle.dense_mask(N, N, *vecs)
+        perm = r.permutation(nch)
+        total = np.zeros_like(glob)
+        for rank in range(nch // 2):
+            ids = sorted(perm[2 * rank: 2 * rank + 2])
+            starts, lens = [c * chunk for c in ids], [chunk, chunk]
+            loc = [oracle.localize(v, starts, lens) for v in vecs]
+            pr = oracle.kv_chunk_pairs(2 * chunk, N, cl, *loc)
+            rows = np.concatenate([np.arange(s, s + chunk) for s in starts])
+            seen = (~dense[rows]).reshape(rows.size, -1, cl).any(axis=(0, 2))
+            np.testing.assert_array_equal(pr > 0, seen)
+            pruned += int((pr == 0).sum())
+            total += pr
+        np.testing.assert_array_equal(total, glob)
+        assert glob.sum() == oracle.count_unmasked_dense(N, N, *vecs)
+    assert pruned > 0  # the cases include chunks some ranks never need

@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--masks", default=None, help="comma list of mask names (default: the config's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the phases eagerly instead of graph replays")
     return ap.parse_args()
 
 
@@ -276,49 +277,82 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
-    def step(rec=None):
-        launches = 0
-        loc_in = [vec_dev[0][c] for c in range(4)]
-        fm.fm_localize(loc_in, loc_starts, loc_lens)
-        launches += 1
-        for mi in range(len(wl["masks"])):
-            vt = vec_dev[mi]
-            if rec is not None:
-                rec["m0"][mi].record(stream)
-            meta = fm.fm_build_mask_meta(*vt, n_q=n)
-            if rec is not None:
-                rec["f0"][mi].record(stream)
-            fm.fm_attn_fwd(q, k, v, meta, vt, scale, o=o, lse=lse)
-            if rec is not None:
-                rec["f1"][mi].record(stream)
-            fm.fm_attn_bwd(q, k, v, o, lse, do, meta, vt, scale, dq=dq, dk=dk, dv=dv, ws=bws)
-            if rec is not None:
-                rec["b1"][mi].record(stream)
-            launches += 2 + 1 + 3
-        return launches
+    n_loc = [sum(x) for x in loc_lens]
+    nm = len(wl["masks"])
+    last = {"meta": [None] * nm}
+    state = {}
+
+    # The step as an ordered list of phases (kind, callable, kernel launches): localization of the
+    # simulated ranks, their KV-chunk pair counts, then metadata, forward and backward per mask.
+    def p_loc():
+        state["loc"] = fm.fm_localize([vec_dev[0][c] for c in range(4)], loc_starts, loc_lens)
+
+    def p_kv():
+        last["pairs"] = fm.fm_kv_chunk_pairs(state["loc"], n_loc, chunk)
+
+    phases = [("localize", p_loc, 1), ("kv_chunk_pairs", p_kv, 1)]
+    for mi in range(nm):
+        def p_meta(mi=mi):
+            last["meta"][mi] = fm.fm_build_mask_meta(*vec_dev[mi], n_q=n)
+
+        def p_fwd(mi=mi):
+            fm.fm_attn_fwd(q, k, v, last["meta"][mi], vec_dev[mi], scale, o=o, lse=lse)
+
+        def p_bwd(mi=mi):
+            fm.fm_attn_bwd(q, k, v, o, lse, do, last["meta"][mi], vec_dev[mi], scale, dq=dq, dk=dk, dv=dv, ws=bws)
+        phases += [("meta", p_meta, 3), ("fwd", p_fwd, 1), ("bwd", p_bwd, 3)]
+    launches_per_step = sum(x[2] for x in phases)
 
     import torch.distributed as dist
     for _ in range(args.warmup):
-        step()
+        for _, fn, _ in phases:
+            fn()
     torch.cuda.synchronize()
+    # Each phase is captured in its own CUDA graph (the host cost of the ctypes calls and output
+    # allocations would otherwise leave the GPU idle between the small kernels); events between
+    # the graph launches time the phases.
+    runners, graphs_used = [fn for _, fn, _ in phases], False
+    if not args.no_graph:
+        try:
+            graphs = []
+            for _, fn, _ in phases:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    fn()
+                graphs.append(g)
+            for g in graphs:  # one replay of the whole step before timing
+                g.replay()
+            torch.cuda.synchronize()
+            runners, graphs_used = [g.replay for g in graphs], True
+        except Exception as exc:  # keep the eager launches (same kernels)
+            print(f"bench: graph capture failed ({exc}); timing eager launches", file=sys.stderr)
     if world > 1:
         dist.barrier()
-    nm = len(wl["masks"])
-    recs = [{key: [ev() for _ in range(nm)] for key in ("m0", "f0", "f1", "b1")} for _ in range(args.steps)]
-    starts, ends = [ev() for _ in range(args.steps)], [ev() for _ in range(args.steps)]
+
+    def step(evs=None):
+        for i, run in enumerate(runners):
+            run()
+            if evs is not None:
+                evs[i + 1].record(stream)
+        return launches_per_step
+
+    step_ev = [[ev() for _ in range(len(phases) + 1)] for _ in range(args.steps)]
     launches = 0
     with ClockSampler(local_rank) as clk:
         torch.cuda.synchronize()
         for s in range(args.steps):
             flush.fill_(s & 0xFF)  # L2 flush between steps, outside the step events
-            starts[s].record(stream)
-            launches += step(recs[s])
-            ends[s].record(stream)
+            step_ev[s][0].record(stream)
+            launches += step(step_ev[s])
         torch.cuda.synchronize()
-    step_ms = [starts[s].elapsed_time(ends[s]) for s in range(args.steps)]
-    fwd_ms = sum(recs[s]["f0"][m].elapsed_time(recs[s]["f1"][m]) for s in range(args.steps) for m in range(nm))
-    bwd_ms = sum(recs[s]["f1"][m].elapsed_time(recs[s]["b1"][m]) for s in range(args.steps) for m in range(nm))
-    meta_ms = sum(recs[s]["m0"][m].elapsed_time(recs[s]["f0"][m]) for s in range(args.steps) for m in range(nm))
+    step_ms = [step_ev[s][0].elapsed_time(step_ev[s][-1]) for s in range(args.steps)]
+
+    def phase_ms(kind):
+        return sum(step_ev[s][i].elapsed_time(step_ev[s][i + 1]) for s in range(args.steps)
+                   for i, ph in enumerate(phases) if ph[0] == kind)
+
+    fwd_ms, bwd_ms, meta_ms = phase_ms("fwd"), phase_ms("bwd"), phase_ms("meta")
+    loc_ms, kvc_ms = phase_ms("localize"), phase_ms("kv_chunk_pairs")
     total_ms = sum(step_ms)
     total_ms, fwd_ms, bwd_ms = reduce_max([total_ms, fwd_ms, bwd_ms], world, dev)
     steps = args.steps
@@ -361,6 +395,31 @@ def run_ours(args, rank, world, local_rank):
     assert fm.fm_get_device_status() == 0, "device-side timeout during the bench"
 
     burst, sustained, hbm, src = peaks()
+
+    def bw(nbytes, ms_total, calls):
+        us = ms_total * 1e3 / calls
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us_per_launch": round(us, 2), "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1),
+                "frac_of_hbm": round(gbs / hbm, 4)}
+
+    # algorithmic bytes of the integer passes (untimed bookkeeping after the timed region)
+    T = n // 128
+    meta_bytes = 0
+    for mt in last["meta"]:
+        ent = int(mt.row_count.sum().item() + mt.col_count.sum().item())
+        meta_bytes += B * (16 * n + 32 * T + T * T + 8 * T + 4 * (T // 2 + T)) + 4 * ent
+    meta_bytes /= nm
+    R = len(loc_starts)
+    pairs = last["pairs"]
+    rank_work = pairs.sum(dim=(1, 2, 3)).double()
+    integer_passes = {
+        "meta": dict(bw(meta_bytes, meta_ms, steps * nm), note="minmax + lists + dispatch order, one call per mask"),
+        "localize": dict(bw(16 * B * n * (1 + R), loc_ms, steps), ranks=R),
+        "kv_chunk_pairs": dict(bw(16 * B * n * R + 8 * pairs.numel(), kvc_ms, steps), ranks=R,
+                               chunks_pruned=int((pairs == 0).sum().item()), chunks=int(pairs.numel()),
+                               rank_work_max_over_mean=round(float(rank_work.max() / rank_work.mean()), 4)),
+        "batched_n262144_r16": aux_localize(fm, torch, dev, stream, hbm),
+    }
     fwd_tf = flops_fwd * steps / (fwd_ms * 1e-3) / 1e12
     bwd_tf = flops_bwd * steps / (bwd_ms * 1e-3) / 1e12
     dominant = "bwd_kernel" if bwd_ms >= fwd_ms else "fwd_kernel"
@@ -374,6 +433,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": wl["desc"], "B": B, "H": H, "seq_len": n, "head_dim": D,
                    "masks": [m for m, _ in wl["masks"]], "unmasked_pairs_per_head": U,
                    "localize": "8 simulated ranks, dual-chunk, 16 chunks", "parallelism": f"replicas x{world}",
+                   "launch": "one CUDA graph per phase, replayed" if graphs_used else "eager",
                    "l2": "flushed between steps (256 MiB write outside the step events); inputs 256 MiB > L2"},
         "fwd": {"effective_tflops": round(fwd_tf, 2), "frac_of_measured_burst": round(fwd_tf / burst, 4),
                 "frac_of_2250_nominal": round(fwd_tf / 2250.0, 4), "ms_per_step": round(fwd_ms / steps, 4)},
@@ -381,6 +441,7 @@ def run_ours(args, rank, world, local_rank):
                 "frac_of_2250_nominal": round(bwd_tf / 2250.0, 4), "ms_per_step": round(bwd_ms / steps, 4),
                 "note": "includes the D_i preprocess and dQ convert kernels"},
         "meta_ms_per_step": round(meta_ms / steps, 4),
+        "integer_passes": integer_passes,
         "roofline": {"bound": "tensor", "kernel": dominant, "achieved": round(ach, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(ach / peak, 4),
                      "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)",
@@ -388,6 +449,48 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
     }
     return line, wl
+
+
+def aux_localize(fm, torch, dev, stream, hbm, reps=20):
+    """The batched form of the integer passes at the localization workload's size: causal documents
+    (L ~ U[4096, 65536]) over N = 262144 keys, 32 chunks of 8192 dealt to 16 simulated ranks (rank r
+    gets chunks r and 31 - r), all ranks in one launch; then the per-rank KV-chunk pair counts."""
+    N, nch = 262144, 32
+    chunk, R = N // nch, nch // 2
+    spec = synth.mask_causal_document(N, synth.draw_docs(synth.Rng(5000), N, 4096, 65536))
+    vt = [torch.from_numpy(np.ascontiguousarray(x[None, None])).to(dev) for x in spec.vectors()]
+    starts = [[r * chunk, (nch - 1 - r) * chunk] for r in range(R)]
+    lens = [[chunk, chunk]] * R
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    loc = fm.fm_localize(vt, starts, lens)
+    pairs = fm.fm_kv_chunk_pairs(loc, [2 * chunk] * R, chunk)
+    g_loc, g_kv = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()  # reps back-to-back launches each
+    with torch.cuda.graph(g_loc):
+        for _ in range(reps):
+            fm.fm_localize(vt, starts, lens, out=loc)
+    with torch.cuda.graph(g_kv):
+        for _ in range(reps):
+            fm.fm_kv_chunk_pairs(loc, [2 * chunk] * R, chunk, out=pairs)
+    g_loc.replay()
+    g_kv.replay()
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    g_loc.replay()
+    ev[1].record(stream)
+    g_kv.replay()
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    out = {}
+    for name, ms, nbytes in (("localize", ev[0].elapsed_time(ev[1]), 16 * N * (1 + R)),
+                             ("kv_chunk_pairs", ev[1].elapsed_time(ev[2]), 16 * N * R + 8 * pairs.numel())):
+        us = ms * 1e3 / reps
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"us_per_launch": round(us, 2), "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / hbm, 4)}
+    work = pairs.sum(dim=(1, 2, 3)).double()
+    out["kv_chunk_pairs"].update(chunks_pruned=int((pairs == 0).sum().item()), chunks=int(pairs.numel()),
+                                 rank_work_max_over_mean=round(float(work.max() / work.mean()), 4))
+    return out
 
 
 def run_reference(args):

@@ -140,6 +140,29 @@ fm_status fm_localize(int32_t B, int32_t Hm, int32_t N, const int32_t* const in[
                       const int32_t* chunk_start, const int32_t* chunk_len, int32_t* const out[4],
                       fm_stream_t stream);
 
+/*
+ * KV-chunk pruning for context-parallel ranks (explainer, across-ranks paragraph:
+ * the forward all-gather skips key-value chunks that are fully masked).  For
+ * each rank r, with n_loc[r] local query rows and the localized vectors
+ * fm_localize wrote, and key chunk c = keys [c * chunk_len, min((c+1) * chunk_len, N)):
+ *     pairs[r, b, hm, c] = sum over keys j of chunk c of
+ *                          n_loc[r] - |([LTS_j, LTE_j) u [UTS_j, UTE_j)) n [0, n_loc[r])|,
+ * the number of unmasked (local row, key) pairs.  A chunk with pairs == 0 is
+ * pruned: no local query attends to any of its keys, so the rank never needs
+ * its K/V.  Summed over chunks it is the rank's attention work (the quantity a
+ * sparsity-aware balancer equalises).  Exact integer counts.
+ *   B, Hm, N     vector shape per rank [B, Hm, N]
+ *   R            ranks, 1 <= R <= 256, R * B * Hm <= 65535
+ *   vec[4]       host array of 4 device pointers, each [R, B, Hm, N] int32
+ *                (NULL = canonical empty: LTS = LTE = n_loc[r], UTS = UTE = 0)
+ *   n_loc        host int32 [R], local query rows of each rank (>= 0)
+ *   chunk_len    keys per chunk (>= 1); n_chunks = ceil(N / chunk_len)
+ *   pairs        device int64 [R, B, Hm, n_chunks], 8-byte aligned
+ * Errors: FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED (R * B * Hm > 65535), FM_ERR_CUDA.
+ */
+fm_status fm_kv_chunk_pairs(int32_t B, int32_t Hm, int32_t N, int32_t R, const int32_t* const vec[4],
+                            const int32_t* n_loc, int32_t chunk_len, int64_t* pairs, fm_stream_t stream);
+
 /* Attention problem.  q, k, v are device pointers (bf16, layouts above). */
 typedef struct {
   int32_t B, H, n_q, n_k, D;

@@ -9,6 +9,7 @@ cannot be loaded, ``lib()`` raises.
 Entry points (same names as the C ABI):
   fm_build_mask_meta(lts, lte, uts, ute, n_q)      -> MaskMeta
   fm_localize(vecs, chunk_start, chunk_len)         -> 4 tensors [R, B, Hm, N]
+  fm_kv_chunk_pairs(loc_vecs, n_loc, chunk_len)     -> int64 [R, B, Hm, n_chunks]
   fm_attn_fwd(q, k, v, meta, vecs, scale)           -> (o, lse)
   fm_attn_bwd(q, k, v, o, lse, do, meta, vecs, scale) -> (dq, dk, dv)
 """
@@ -70,6 +71,8 @@ def lib():
         L.fm_localize.argtypes = [i32, i32, i32, VecArray, i32, i32, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.POINTER(ctypes.c_int32), VecArray, vp]
         L.fm_localize.restype = ctypes.c_int
+        L.fm_kv_chunk_pairs.argtypes = [i32, i32, i32, i32, VecArray, ctypes.POINTER(ctypes.c_int32), i32, vp, vp]
+        L.fm_kv_chunk_pairs.restype = ctypes.c_int
         L.fm_attn_fwd.argtypes = [ctypes.POINTER(AttnArgs), ctypes.POINTER(MaskMetaC), VecArray, vp, vp, vp]
         L.fm_attn_fwd.restype = ctypes.c_int
         L.fm_attn_bwd_workspace_bytes.argtypes = [ctypes.POINTER(AttnArgs)]
@@ -155,19 +158,36 @@ def fm_build_mask_meta(lts, lte, uts, ute, n_q: int, stream=None) -> MaskMeta:
     return MaskMeta(d, ws, c)
 
 
-def fm_localize(vecs, chunk_start, chunk_len, stream=None):
+def fm_localize(vecs, chunk_start, chunk_len, out=None, stream=None):
     """vecs: 4 int32 CUDA tensors [B, Hm, N]; chunk_start / chunk_len: [R, C] host ints.
-    Returns 4 int32 tensors [R, B, Hm, N]."""
+    Returns 4 int32 tensors [R, B, Hm, N] (written into `out` when given)."""
     import numpy as np
     cs = np.ascontiguousarray(np.asarray(chunk_start, dtype=np.int32))
     cl = np.ascontiguousarray(np.asarray(chunk_len, dtype=np.int32))
     R, C = cs.shape
     B, Hm, N = vecs[0].shape
-    outs = [torch.empty((R, B, Hm, N), dtype=torch.int32, device=vecs[0].device) for _ in range(4)]
+    outs = out if out is not None else [torch.empty((R, B, Hm, N), dtype=torch.int32, device=vecs[0].device)
+                                        for _ in range(4)]
     _check(lib().fm_localize(B, Hm, N, _vecs(vecs), R, C, cs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                              cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _vecs(outs), _stream(stream)),
            "fm_localize")
     return outs
+
+
+def fm_kv_chunk_pairs(loc_vecs, n_loc, chunk_len: int, out=None, stream=None):
+    """loc_vecs: 4 int32 CUDA tensors [R, B, Hm, N] (fm_localize's output; None = canonical empty);
+    n_loc: R host ints.  Returns int64 [R, B, Hm, ceil(N / chunk_len)] unmasked-pair counts per KV chunk."""
+    import numpy as np
+    ref = next(v for v in loc_vecs if v is not None)
+    R, B, Hm, N = ref.shape
+    nl = np.ascontiguousarray(np.asarray(n_loc, dtype=np.int32))
+    if nl.shape != (R,):
+        raise FmError(FM_ERR_INVALID_ARG, "fm_kv_chunk_pairs: n_loc must hold one row count per rank")
+    if out is None:
+        out = torch.empty((R, B, Hm, -(-N // chunk_len)), dtype=torch.int64, device=ref.device)
+    _check(lib().fm_kv_chunk_pairs(B, Hm, N, R, _vecs(loc_vecs), nl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                   int(chunk_len), _ptr(out), _stream(stream)), "fm_kv_chunk_pairs")
+    return out
 
 
 def _args(q, k, v, scale) -> AttnArgs:

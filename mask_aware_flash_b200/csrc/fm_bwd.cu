@@ -700,9 +700,7 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.group = dispatch_group(p.H, (double)a->n_q * D * (2 * S::kElem + 4));  // Q, dO, fp32 dQ accumulator
   p.scale = a->scale;
   p.scale_log2 = a->scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(bwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
-      cudaSuccess)
-    return FM_ERR_CUDA;
+  if (!smem_opt_in<bwd_kernel<D, F32>>(S::kAlloc)) return FM_ERR_CUDA;
   bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
   bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (a->n_q / 64)), 256, 0, stream>>>(
       acc, dq, a->B, a->H, a->n_q, a->scale);

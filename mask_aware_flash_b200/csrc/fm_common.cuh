@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "fm.h"
 
 namespace fm {
@@ -490,6 +492,19 @@ __device__ __forceinline__ int ld_nc_i32(const int32_t* p) {
 // ---------------------------------------------------------------------------
 namespace fm {
 int* device_status_ptr();  // per-device status word; nullptr on failure
+// Raises a kernel's dynamic shared-memory limit once per device (then never again,
+// so later launches, e.g. inside a CUDA-graph capture, make no attribute calls).
+template <auto kernel>  // one instance (and one flag word) per kernel
+bool smem_opt_in(int bytes) {
+  static std::atomic<uint64_t> done{0};  // one bit per device (devices 0..63)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done.fetch_or(bit, std::memory_order_release);
+  return true;
+}
 // Heads whose CTAs an attention kernel dispatches together: as many as keep the
 // per-head bytes that all CTAs of a head re-read within 32 MiB of L2 (at least 1,
 // at most H).

@@ -584,9 +584,7 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.n_pairs = (p.T_q + 1) / 2;
   p.group = dispatch_group(p.H, 2.0 * a->n_k * D * S::kElem);
   p.scale_log2 = a->scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(fwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) !=
-      cudaSuccess)
-    return FM_ERR_CUDA;
+  if (!smem_opt_in<fwd_kernel<D, F32>>(S::kAlloc)) return FM_ERR_CUDA;
   fwd_kernel<D, F32><<<dim3(p.group * p.n_pairs, (p.H + p.group - 1) / p.group, p.B), kFwdThreads, S::kAlloc, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }

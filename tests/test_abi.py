@@ -146,3 +146,22 @@ def test_no_oracle_import_in_library():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "fm_oracle" not in txt, f
+
+
+def test_kv_chunk_pairs_rejects_bad_args(L):
+    import numpy as np
+    vec = fm.VecArray(0x10000, 0x20000, 0x30000, 0x40000)
+    nl = np.array([64, 64], np.int32)
+    p_nl = nl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    out = ctypes.c_void_p(0x50000)
+    assert L.fm_kv_chunk_pairs(1, 1, 256, 2, vec, p_nl, 0, out, None) == fm.FM_ERR_INVALID_ARG  # chunk_len
+    assert L.fm_kv_chunk_pairs(1, 1, 256, 0, vec, p_nl, 64, out, None) == fm.FM_ERR_INVALID_ARG  # no ranks
+    assert L.fm_kv_chunk_pairs(1, 1, 256, 2, vec, p_nl, 64, ctypes.c_void_p(0x50004), None) == \
+        fm.FM_ERR_INVALID_ARG  # misaligned int64 output
+    assert L.fm_kv_chunk_pairs(1, 1, 256, 2, vec, None, 64, out, None) == fm.FM_ERR_INVALID_ARG
+    bad = np.array([64, -1], np.int32)
+    assert L.fm_kv_chunk_pairs(1, 1, 256, 2, vec, bad.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), 64, out,
+                               None) == fm.FM_ERR_INVALID_ARG
+    many = np.full(256, 64, np.int32)
+    assert L.fm_kv_chunk_pairs(300, 1, 256, 256, vec, many.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), 64, out,
+                               None) == fm.FM_ERR_UNSUPPORTED  # 256 ranks x 300 rows > 65535

@@ -171,6 +171,14 @@ def test_localization_262144_16_ranks(fm):
         got = loc[c][:, 0, 0, keys].cpu().numpy()
         for r in range(R):
             np.testing.assert_array_equal(got[r], oracle.localize(spec.vectors()[c][keys], starts[r], lens[r]))
+    # KV-chunk pruning: per-rank unmasked pairs per KV chunk, bit-exact; over the ranks (which
+    # partition the rows) they add up to the global mask's pairs per chunk
+    pairs = fm.fm_kv_chunk_pairs(loc, [2 * chunk] * R, chunk).cpu().numpy()[:, 0, 0]
+    for r in range(R):
+        lv = [x[r, 0, 0].cpu().numpy() for x in loc]
+        np.testing.assert_array_equal(pairs[r], oracle.kv_chunk_pairs(2 * chunk, N, chunk, *lv))
+    np.testing.assert_array_equal(pairs.sum(0), oracle.kv_chunk_pairs(N, N, chunk, *spec.vectors()))
+    assert (pairs == 0).sum() > 0  # documents: every rank skips some KV chunks
     for r in range(R):
         rows = torch.cat([torch.arange(s, s + chunk) for s in starts[r]]).cuda()
         lv = [x[r].contiguous() for x in loc]

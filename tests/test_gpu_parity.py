@@ -147,6 +147,36 @@ def test_localize_bitexact(fm):
                 np.testing.assert_array_equal(got[rr, b, 0], exp)
 
 
+def test_kv_chunk_pairs_bitexact(fm):
+    """Per-rank unmasked pairs per KV chunk (KV-chunk pruning) on localized vectors: bit-exact
+    against the oracle for random vectors and a document mask, a ragged last chunk, null vectors,
+    and ranks owning different numbers of rows."""
+    N, nch = 4096, 16
+    chunk = N // nch
+    r = np.random.default_rng(19)
+    vecs = [r.integers(-100, N + 100, (2, 1, N)).astype(np.int32) for _ in range(4)]
+    spec = synth.make_family("causal_document", N, 13)
+    for c in range(4):
+        vecs[c][1, 0] = spec.vectors()[c]
+    # 5 ranks: dual chunks, a single chunk and three chunks
+    starts = [[0, 15 * chunk], [chunk, 14 * chunk], [2 * chunk, 13 * chunk], [3 * chunk, 5 * chunk],
+              [6 * chunk, 9 * chunk]]
+    lens = [[chunk, chunk], [chunk, chunk], [chunk, chunk], [2 * chunk, 4 * chunk], [3 * chunk, 4 * chunk]]
+    n_loc = [sum(x) for x in lens]
+    loc = fm.fm_localize([torch.from_numpy(v).cuda() for v in vecs], starts, lens)
+    for cl in (chunk, 1000):  # aligned chunks and a ragged last chunk
+        got = fm.fm_kv_chunk_pairs(loc, n_loc, cl).cpu().numpy()
+        for rr in range(len(starts)):
+            for b in range(2):
+                lv = [x[rr, b, 0].cpu().numpy() for x in loc]
+                np.testing.assert_array_equal(got[rr, b, 0], oracle.kv_chunk_pairs(n_loc[rr], N, cl, *lv))
+    # null vectors = canonical empty: every pair of the rank is unmasked
+    nul = fm.fm_kv_chunk_pairs([None, None, None, loc[3]], n_loc, chunk).cpu().numpy()
+    for rr in range(len(starts)):
+        lv = loc[3][rr, 0, 0].cpu().numpy()
+        np.testing.assert_array_equal(nul[rr, 0, 0], oracle.kv_chunk_pairs(n_loc[rr], N, chunk, None, None, None, lv))
+
+
 # ---------------------------------------------------------------------------- attention
 def _run_attention(fm, B, H, n_q, n_k, D, vecs_np, Hm, seed, scale=None, bwd=True):
     scale = 1.0 / math.sqrt(D) if scale is None else scale

@@ -105,18 +105,9 @@ __device__ __forceinline__ void transpose64_f32(uint8_t* t, int tid) {
   }
 }
 
-// AND of a flag over the 128 drain threads (named barrier 1): every thread reaches it after its own
-// bounded wait, so the threads leave or enter a transpose (which synchronises on barrier 1) together.
-__device__ __forceinline__ bool all_drain_threads(bool v) {
-  int r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
-      "selp.s32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((int)v)
-      : "memory");
-  return r != 0;
-}
+// The 128 drain threads leave or enter a transpose (which synchronises on named barrier 1)
+// together: each votes after its own bounded wait.
+__device__ __forceinline__ bool all_drain_threads(bool v) { return named_bar_and(1, 128, v); }
 
 // K [128 keys][64 d] -> K^T [64 d][128 keys], both fp32 with 128-byte swizzle, by 128 threads.
 __device__ __forceinline__ void transpose_k_f32(const uint8_t* k, uint8_t* kt, int tid) {

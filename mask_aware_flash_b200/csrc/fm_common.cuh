@@ -123,6 +123,17 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Named barrier that also returns the AND of `v` over the `count` participating threads.
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool v) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((int)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
 // generic-proxy smem writes -> visible to the async proxy (tensor core reads)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -439,10 +450,11 @@ __device__ __forceinline__ uint32_t interval_bits32(int32_t start, int32_t end, 
   return b > a ? ((0xFFFFFFFFu >> (32 - b)) & (0xFFFFFFFFu << a)) : 0u;
 }
 
-// Transpose of four 32 x 32 bit matrices held one row per lane: on return bit l of
+// Transpose of N 32 x 32 bit matrices held one row per lane: on return bit l of
 // lane r's word w[j] is bit r of lane l's word w[j] on entry.  Five butterfly
 // stages; at stage s, lanes l and l ^ s swap the off-diagonal s x s blocks.
-__device__ __forceinline__ void bit_transpose32x4(uint32_t (&w)[4], int lane) {
+template <int N>
+__device__ __forceinline__ void bit_transpose32(uint32_t (&w)[N], int lane) {
   constexpr uint32_t kLow[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
 #pragma unroll
   for (int st = 0; st < 5; ++st) {
@@ -450,7 +462,7 @@ __device__ __forceinline__ void bit_transpose32x4(uint32_t (&w)[4], int lane) {
     const bool upper = (lane & s) != 0;
     const uint32_t keep = upper ? ~kLow[st] : kLow[st];  // bits this lane keeps
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < N; ++j) {
       const uint32_t y = __shfl_xor_sync(0xffffffffu, w[j], s);
       const uint32_t t = upper ? (y >> s) : (y << s);
       w[j] = (w[j] & keep) | (t & ~keep);

@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int32_t uts = has[2] ? mv[2 * kTile + c] : 0, ute = has[3] ? mv[3 * kTile + c] : 0;
             mw[jb] = interval_bits32(lts, lte, w0) | interval_bits32(uts, ute, w0);
           }
-          bit_transpose32x4(mw, lane);
+          bit_transpose32<4>(mw, lane);
 #pragma unroll
           for (int jb = 0; jb < 4; ++jb) {
             if (__any_sync(0xffffffffu, mw[jb] != 0u)) {

@@ -253,6 +253,18 @@ fm_status fm_get_device_status(fm_stream_t stream);
 /* Static description of a status code. */
 const char* fm_status_string(fm_status s);
 
+/*
+ * Self-test of the bounded-wait path (no counterpart in the paper).  Every wait in
+ * the kernels gives up after 2 s, records FM_ERR_DEVICE_TIMEOUT in the per-device
+ * status word and lets its kernel return, so a stuck pipeline surfaces as a status
+ * instead of a hung GPU.  This call enqueues one kernel whose only wait is on a
+ * barrier nothing completes: about 2 s later it has recorded the timeout, which the
+ * next fm_get_device_status(stream) returns (and clears).  Nothing faults; the
+ * context stays usable.
+ * Errors: FM_ERR_CUDA (launch failed).
+ */
+fm_status fm_selftest_wait_timeout(fm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -82,6 +82,8 @@ def lib():
         L.fm_attn_bwd.restype = ctypes.c_int
         L.fm_get_device_status.argtypes = [vp]
         L.fm_get_device_status.restype = ctypes.c_int
+        L.fm_selftest_wait_timeout.argtypes = [vp]
+        L.fm_selftest_wait_timeout.restype = ctypes.c_int
         L.fm_status_string.argtypes = [ctypes.c_int]
         L.fm_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -228,6 +230,12 @@ def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=No
     _check(lib().fm_attn_bwd(ctypes.byref(a), ctypes.byref(meta.c), _vecs(vecs), _ptr(o), _ptr(lse), _ptr(do),
                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)), "fm_attn_bwd")
     return dq, dk, dv
+
+
+def fm_selftest_wait_timeout(stream=None):
+    """Enqueue the bounded-wait self-test (a wait that runs out after ~2 s and records
+    FM_ERR_DEVICE_TIMEOUT for the next fm_get_device_status)."""
+    _check(lib().fm_selftest_wait_timeout(_stream(stream)), "fm_selftest_wait_timeout")
 
 
 def fm_get_device_status(stream=None) -> int:

@@ -79,9 +79,31 @@ bool encode_tmap_f32_4d(CUtensorMap* map, const void* base, uint64_t D, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// One CTA waits on an mbarrier that nothing arrives on.  The bounded wait gives
+// up after kTimeoutNs and records FM_ERR_DEVICE_TIMEOUT (site 0x7E57) in the
+// device status word; the kernel then returns normally.
+__global__ void selftest_wait_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(smem_u32(&bar), 0, &abort_flag)) record_failure(status, &abort_flag, 0x7E57);
+}
+
 }  // namespace fm
 
 extern "C" {
+
+fm_status fm_selftest_wait_timeout(fm_stream_t stream) {
+  int* st = fm::device_status_ptr();
+  if (!st) return FM_ERR_CUDA;
+  fm::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(st);
+  return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
+}
 
 const char* fm_status_string(fm_status s) {
   switch (s) {

@@ -53,7 +53,7 @@ typedef struct CUstream_st* fm_stream_t; /* identical to cudaStream_t */
 typedef enum {
   FM_OK = 0,
   FM_ERR_INVALID_ARG = 1,     /* a size, pointer, alignment or ordering rule is broken */
-  FM_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. n not a multiple of 128) */
+  FM_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. n_k not a multiple of 4) */
   FM_ERR_WORKSPACE = 3,       /* workspace pointer NULL/misaligned or ws_bytes too small */
   FM_ERR_CUDA = 4,            /* a CUDA runtime/driver call or launch failed */
   FM_ERR_DEVICE_TIMEOUT = 5   /* a kernel's bounded wait ran out (see fm_get_device_status) */
@@ -179,7 +179,9 @@ typedef struct {
  * LSE_i = ln sum_{j in U_i} exp(scale q_i.k_j); a row with U_i empty gets
  * O_i = 0 and LSE_i = -inf.  Only non-skip key tiles (meta row lists) are read;
  * the row-interval test runs on partial tiles only.
- *   a      host struct; n_q, n_k multiples of 128; D in {64, 128}; dtype 0, or 1 with D = 64;
+ *   a      host struct; n_q >= 1 any length, n_k >= 1 a multiple of 4 (ragged lengths: the last
+ *          tiles are zero-filled past n and the last key tile always runs the interval test);
+ *          at most 4096 tiles each way; D in {64, 128}; dtype 0, or 1 with D = 64;
  *          scale > 0 and finite.
  *   meta   host struct from fm_build_mask_meta with d = {B, Hm, n_q, n_k, 128, 128}.
  *   vec[4] host array of the 4 device vector pointers meta was built from

@@ -47,6 +47,7 @@ struct BwdParams {
   void* dv;
   int* status;
   int B, H, Hm, n_q, n_k, T_q, T_k;
+  int n_q_pad;                 // n_q rounded up to whole query tiles (row stride of lse2, dvec, dq_acc)
   int group;                   // heads dispatched together
   float scale, scale_log2;
 };
@@ -216,8 +217,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_4d(q_s + st * S::kQStage + c * 8192, &tm_q, fb, c * kAtomElems, h, q0, b);
           tma_load_4d(do_s + st * S::kQStage + c * 8192, &tm_do, fb, c * kAtomElems, h, q0, b);
         }
-        bulk_load(smem_u32(stats + st * 2 * kBQ), p.lse2 + bh * p.n_q + q0, kBQ * 4, fb);
-        bulk_load(smem_u32(stats + st * 2 * kBQ + kBQ), p.dvec + bh * p.n_q + q0, kBQ * 4, fb);
+        bulk_load(smem_u32(stats + st * 2 * kBQ), p.lse2 + bh * p.n_q_pad + q0, kBQ * 4, fb);
+        bulk_load(smem_u32(stats + st * 2 * kBQ + kBQ), p.dvec + bh * p.n_q_pad + q0, kBQ * 4, fb);
       }
     }
   } else if (warp == 13) {
@@ -357,8 +358,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int64_t j = (int64_t)kt * kTile + r;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const int64_t voff = bhm * p.n_k + j;
-    const int32_t lts = p.vec[0] ? __ldg(p.vec[0] + voff) : p.n_q, lte = p.vec[1] ? __ldg(p.vec[1] + voff) : p.n_q;
-    const int32_t uts = p.vec[2] ? __ldg(p.vec[2] + voff) : 0, ute = p.vec[3] ? __ldg(p.vec[3] + voff) : 0;
+    const bool no_key = j >= p.n_k;  // past a ragged n_k: a zero-filled key row, masked for every query
+    const int32_t lts = (p.vec[0] && !no_key) ? __ldg(p.vec[0] + voff) : p.n_q;
+    const int32_t lte = (p.vec[1] && !no_key) ? __ldg(p.vec[1] + voff) : p.n_q;
+    const int32_t uts = (p.vec[2] && !no_key) ? __ldg(p.vec[2] + voff) : 0;
+    const int32_t ute = (p.vec[3] && !no_key) ? __ldg(p.vec[3] + voff) : 0;
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
       const int st = i % NS, bi = i % NDS, sb = i & 1;  // Q/dO stage, dS^T buffer, S^T buffer
@@ -376,7 +380,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float4* l2 = reinterpret_cast<const float4*>(stats + st * 2 * kBQ + c0);
       const float4* dd = reinterpret_cast<const float4*>(stats + st * 2 * kBQ + kBQ + c0);
       // row-interval test (partial tiles only) as a mask of this key's masked queries
-      const uint32_t mbits = partial ? (interval_bits32(lts, lte, q0) | interval_bits32(uts, ute, q0)) : 0u;
+      const uint32_t mbits =
+          no_key ? 0xFFFFFFFFu : (partial ? (interval_bits32(lts, lte, q0) | interval_bits32(uts, ute, q0)) : 0u);
       const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
       uint32_t pk[F32 ? 32 : 16], dk[F32 ? 32 : 16];  // bf16 pairs or tf32-rounded fp32
 #pragma unroll
@@ -445,7 +450,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // dP^T have read the stage)
     const int d = threadIdx.x - 256;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-    float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q * D;
+    float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q_pad * D;
     bool ok = true;
     if constexpr (F32) {
       if (nsub > 0) {
@@ -555,7 +560,7 @@ template <int D, bool F32>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ o, const void* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ dvec, float* __restrict__ acc, int B,
-                                                       int H, int n_q) {
+                                                       int H, int n_q, int n_q_pad) {
   const int64_t rows = (int64_t)B * n_q * H;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t < rows) {
@@ -587,15 +592,24 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ 
         }
       }
     }
-    const int64_t out = ((int64_t)b * H + h) * n_q + i;
+    const int64_t out = ((int64_t)b * H + h) * n_q_pad + i;  // rows padded to whole query tiles
     dvec[out] = s;
-    const float l = lse[out];
+    const float l = lse[((int64_t)b * H + h) * n_q + i];
     lse2[out] = (l == kNegInf) ? kPosInf : l * 1.4426950408889634f;
   }
-  // clear the accumulator (B*H*n_q*D floats), grid-stride in float4
+  // padding rows past a ragged n_q: P = 0 there (log2 LSE = +inf), D_i = 0
+  const int pad = n_q_pad - n_q;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  if (pad > 0)
+    for (int64_t k = t; k < (int64_t)B * H * pad; k += stride) {
+      const int64_t row = (k / pad) * n_q_pad + n_q + (k % pad);
+      lse2[row] = kPosInf;
+      dvec[row] = 0.f;
+    }
+  // clear the accumulator (B*H*n_q_pad*D floats), grid-stride in float4
   float4* a4 = reinterpret_cast<float4*>(acc);
-  const int64_t n4 = rows * D / 4;
-  for (int64_t k = t; k < n4; k += (int64_t)gridDim.x * blockDim.x) a4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int64_t n4 = (int64_t)B * H * n_q_pad * D / 4;
+  for (int64_t k = t; k < n4; k += stride) a4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ[b, i, h, :] = scale * acc for one 64-row block per CTA: the block (a
@@ -603,17 +617,18 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ 
 // against bank conflicts), then each thread writes 8 consecutive d of one row.
 template <int D, bool F32>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, void* __restrict__ dq,
-                                                     int B, int H, int n_q, float scale) {
+                                                     int B, int H, int n_q, int n_q_pad, float scale) {
   __shared__ float4 buf[16 * D + 2 * D];  // one float4 of padding per 8
-  const int blocks_per_bh = n_q / 64;
+  const int blocks_per_bh = n_q_pad / 64;
   const int64_t bh = blockIdx.x / blocks_per_bh;
   const int qb = blockIdx.x % blocks_per_bh;
   const int b = (int)(bh / H), h = (int)(bh % H);
-  const float4* src = reinterpret_cast<const float4*>(acc + (bh * n_q + (int64_t)qb * 64) * D);
+  const float4* src = reinterpret_cast<const float4*>(acc + (bh * n_q_pad + (int64_t)qb * 64) * D);
   for (int k = threadIdx.x; k < 16 * D; k += blockDim.x) buf[k + (k >> 3)] = __ldg(src + k);
   __syncthreads();
   for (int w = threadIdx.x; w < 64 * (D / 8); w += blockDim.x) {
     const int q = w / (D / 8), d0 = (w % (D / 8)) * 8;
+    if (qb * 64 + q >= n_q) continue;  // padding rows past a ragged n_q
     const int g = q >> 2, u = q & 3;
     float x[8];
 #pragma unroll
@@ -643,7 +658,7 @@ struct BwdLayout {
 
 BwdLayout bwd_layout(const fm_attn_args* a) {
   BwdLayout L;
-  const size_t rows = (size_t)a->B * a->H * a->n_q;
+  const size_t rows = (size_t)a->B * a->H * (((size_t)a->n_q + kTile - 1) / kTile * kTile);  // padded rows
   L.acc = 0;
   L.lse2 = align256(rows * a->D * 4);
   L.dvec = L.lse2 + align256(rows * 4);
@@ -669,7 +684,7 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
     return FM_ERR_CUDA;
   const int64_t rows = (int64_t)a->B * a->n_q * a->H;
   bwd_prep_kernel<D, F32><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(o, dout, lse, lse2, dvec, acc, a->B,
-      a->H, a->n_q);
+      a->H, a->n_q, (a->n_q + kTile - 1) / kTile * kTile);
   BwdParams p;
   p.col_count = meta->col_count;
   p.col_entries = meta->col_entries;
@@ -686,15 +701,16 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.Hm = meta->d.Hm;
   p.n_q = a->n_q;
   p.n_k = a->n_k;
-  p.T_q = a->n_q / kTile;
-  p.T_k = a->n_k / kTile;
+  p.T_q = (a->n_q + kTile - 1) / kTile;
+  p.T_k = (a->n_k + kTile - 1) / kTile;
+  p.n_q_pad = p.T_q * kTile;
   p.group = dispatch_group(p.H, (double)a->n_q * D * (2 * S::kElem + 4));  // Q, dO, fp32 dQ accumulator
   p.scale = a->scale;
   p.scale_log2 = a->scale * 1.4426950408889634f;
   if (!smem_opt_in<bwd_kernel<D, F32>>(S::kAlloc)) return FM_ERR_CUDA;
   bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
-  bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (a->n_q / 64)), 256, 0, stream>>>(
-      acc, dq, a->B, a->H, a->n_q, a->scale);
+  bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (p.n_q_pad / 64)), 256, 0, stream>>>(
+      acc, dq, a->B, a->H, a->n_q, p.n_q_pad, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

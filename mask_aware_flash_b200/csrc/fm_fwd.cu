@@ -75,17 +75,21 @@ struct FwdSmem {
 // Yields each key tile once with the class it has for each query tile
 // (0 skip, 1 partial, 2 full).  Every role runs its own copy over the same
 // shared-memory lists, so all roles see the same sequence.
+// A key tile that runs past n_k (ragged length) is always treated as partial:
+// its columns beyond n_k hold zero-filled keys that the interval test masks.
 struct MergedList {
   const uint16_t* a;
   const uint16_t* b;
   int na, nb, pa, pb;
+  int ragged_kt;  // index of the key tile that runs past n_k, or -1
   __device__ __forceinline__ bool next(int& kt, int& c0, int& c1) {
     const int ea = pa < na ? a[pa] : INT_MAX, eb = pb < nb ? b[pb] : INT_MAX;
     const int ka = ea >> 1, kb = eb >> 1;
     kt = min(ka, kb);
     if (kt == (INT_MAX >> 1)) return false;
-    c0 = (ka == kt) ? ((ea & 1) ? 1 : 2) : 0;
-    c1 = (kb == kt) ? ((eb & 1) ? 1 : 2) : 0;
+    const bool rag = kt == ragged_kt;
+    c0 = (ka == kt) ? (((ea & 1) || rag) ? 1 : 2) : 0;
+    c1 = (kb == kt) ? (((eb & 1) || rag) ? 1 : 2) : 0;
     pa += (ka == kt);
     pb += (kb == kt);
     return true;
@@ -93,17 +97,18 @@ struct MergedList {
 };
 
 // fp32 path: kind::tf32 MMAs read both operands K-major, so PV needs V^T
-// ([d][key], keys contiguous).  One warp copies a 128-key fp32 V tile from
-// global memory into that layout (128-byte swizzle; four atoms of 32 keys,
+// ([d][key], keys contiguous).  One warp copies a 128-key fp32 V tile (its first
+// `valid` keys; zeros after them) from global memory into that layout (128-byte swizzle; four atoms of 32 keys,
 // D rows of 128 bytes each), rounding to tf32 on the way: element (d, key) sits
 // at (key / 32) * D * 128 + d * 128 + ((((key % 32) / 4) ^ (d % 8)) * 16) + (key % 4) * 4.
 template <int D>
-__device__ __forceinline__ void load_vt_f32(uint8_t* dst, const float* src, int64_t row_stride, int lane) {
+__device__ __forceinline__ void load_vt_f32(uint8_t* dst, const float* src, int64_t row_stride, int valid, int lane) {
   constexpr int kQuads = D / 4;
 #pragma unroll 4
   for (int e = lane; e < kTile * kQuads; e += 32) {
     const int key = e / kQuads, dq = e % kQuads;
-    const float4 x = __ldg(reinterpret_cast<const float4*>(src + key * row_stride) + dq);
+    const float4 x = key < valid ? __ldg(reinterpret_cast<const float4*>(src + key * row_stride) + dq)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);  // past a ragged n_k
     const float xs[4] = {x.x, x.y, x.z, x.w};
     uint8_t* col = dst + (key >> 5) * (D * 128) + (key & 3) * 4;
 #pragma unroll
@@ -139,6 +144,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int32_t* rows1 = rows0 + p.T_k;
   const int n0 = __ldg(p.row_count + bhm * p.T_q + qt0);
   const int n1 = has1 ? __ldg(p.row_count + bhm * p.T_q + qt1) : 0;
+  const int ragged_kt = (p.n_k % kTile) ? p.T_k - 1 : -1;
 
   const uint32_t bar0 = smem_u32(smem + S::kBar);
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -201,7 +207,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       int nvec = 0;
       for (int c = 0; c < 4; ++c) nvec += p.vec[c] ? 1 : 0;
-      MergedList it{list0, list1, n0, n1, 0, 0};
+      MergedList it{list0, list1, n0, n1, 0, 0, ragged_kt};
       int kt, c0, c1, e = 0, mcount = 0;
       bool ok = true;
       while (it.next(kt, c0, c1)) {
@@ -223,11 +229,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             break;
           }
           if (lane == 0) {
-            mbar_arrive_expect_tx(bar(S::M_FULL0 + mb), 512u * nvec);
+            // a ragged last key tile has (n_k - 128 kt) columns, a multiple of 4 (16-byte copies)
+            const uint32_t vbytes = 4u * (uint32_t)min(kTile, p.n_k - kt * kTile);
+            mbar_arrive_expect_tx(bar(S::M_FULL0 + mb), vbytes * nvec);
             for (int c = 0; c < 4; ++c)
               if (p.vec[c])
                 bulk_load(smem_u32(mask_smem + (mb * 4 + c) * kTile), p.vec[c] + bhm * p.n_k + (int64_t)kt * kTile,
-                          512u, bar(S::M_FULL0 + mb));
+                          vbytes, bar(S::M_FULL0 + mb));
           }
           ++mcount;
         }
@@ -237,7 +245,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         if constexpr (F32) {
           load_vt_f32<D>(smem + S::kV + slot * S::kTileBytes,
-                         p.v32 + (((int64_t)b * p.n_k + (int64_t)kt * kTile) * p.H + h) * D, (int64_t)p.H * D, lane);
+                         p.v32 + (((int64_t)b * p.n_k + (int64_t)kt * kTile) * p.H + h) * D, (int64_t)p.H * D,
+                         min(kTile, p.n_k - kt * kTile), lane);
           fence_proxy_async_smem();  // generic-proxy stores, read next by the tensor core
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(S::V_FULL0 + slot));
@@ -259,7 +268,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       constexpr uint32_t kIdescQK = F32 ? idesc_tf32(128, 128, false, false) : idesc_bf16(128, 128, false, false);
       constexpr uint32_t kIdescPV = F32 ? idesc_tf32(128, D, false, false) : idesc_bf16(128, D, false, true);
       constexpr int kPvSteps = kTile / kKStep;  // UMMA K steps over the 128 kv rows
-      MergedList it{list0, list1, n0, n1, 0, 0};
+      MergedList it{list0, list1, n0, n1, 0, 0, ragged_kt};
       int kt, c0, c1, kn, n0c, n1c;
       bool ok = mbar_wait(bar(S::Q_FULL), 0, abort_flag);
       bool has_cur = ok && it.next(kt, c0, c1);
@@ -350,14 +359,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int t = warp >> 2;                   // query tile of this warpgroup
     const int r = threadIdx.x & 127;           // row in tile == TMEM lane
     const int qt = t ? qt1 : qt0;
-    const int64_t i = (int64_t)qt * kTile + r;
+    const int i = qt * kTile + r;  // row (n_q < 2^31)
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + t * 256 + lane_addr, tO = tS + 128;
-    const bool has[4] = {p.vec[0] != nullptr, p.vec[1] != nullptr, p.vec[2] != nullptr, p.vec[3] != nullptr};
+    const uint32_t has = (p.vec[0] ? 1u : 0u) | (p.vec[1] ? 2u : 0u) | (p.vec[2] ? 4u : 0u) | (p.vec[3] ? 8u : 0u);
     float m_run = kNegInf, l_run = 0.f, lq_run = 0.f;
     int j = 0, mcount = 0;
     bool ok = true;
-    MergedList it{list0, list1, n0, n1, 0, 0};
+    MergedList it{list0, list1, n0, n1, 0, 0, ragged_kt};
     int kt, c0, c1;
     const bool live_tile = (t == 0) || has1;
     // A warpgroup without a query tile (odd tile count) still walks the list:
@@ -385,11 +394,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int jb = 0; jb < 4; ++jb) {
             const int c = jb * 32 + lane;
-            const int32_t lts = has[0] ? mv[c] : p.n_q, lte = has[1] ? mv[kTile + c] : p.n_q;
-            const int32_t uts = has[2] ? mv[2 * kTile + c] : 0, ute = has[3] ? mv[3 * kTile + c] : 0;
+            const int32_t lts = (has & 1u) ? mv[c] : p.n_q, lte = (has & 2u) ? mv[kTile + c] : p.n_q;
+            const int32_t uts = (has & 4u) ? mv[2 * kTile + c] : 0, ute = (has & 8u) ? mv[3 * kTile + c] : 0;
             mw[jb] = interval_bits32(lts, lte, w0) | interval_bits32(uts, ute, w0);
           }
           bit_transpose32<4>(mw, lane);
+          if (kt == ragged_kt) {  // columns past a ragged n_k hold no key: masked in every row
+            const int valid = p.n_k - kt * kTile;
+#pragma unroll
+            for (int jb = 0; jb < 4; ++jb) {
+              const int v = valid - jb * 32;  // valid columns of this 32-column block
+              mw[jb] |= v >= 32 ? 0u : (v <= 0 ? 0xFFFFFFFFu : ~((1u << v) - 1u));
+            }
+          }
 #pragma unroll
           for (int jb = 0; jb < 4; ++jb) {
             if (__any_sync(0xffffffffu, mw[jb] != 0u)) {
@@ -543,7 +560,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         bulk_commit_group();
         bulk_wait_group_read0();
       }
-      p.lse[((int64_t)b * p.H + h) * p.n_q + i] = live ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
+      if (i < p.n_q)  // rows past a ragged n_q are computed on zero-filled queries and dropped
+        p.lse[((int64_t)b * p.H + h) * p.n_q + (int64_t)i] = live ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
     }
   }
 
@@ -579,8 +597,8 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.Hm = meta->d.Hm;
   p.n_q = a->n_q;
   p.n_k = a->n_k;
-  p.T_q = a->n_q / kTile;
-  p.T_k = a->n_k / kTile;
+  p.T_q = (a->n_q + kTile - 1) / kTile;
+  p.T_k = (a->n_k + kTile - 1) / kTile;
   p.n_pairs = (p.T_q + 1) / 2;
   p.group = dispatch_group(p.H, 2.0 * a->n_k * D * S::kElem);
   p.scale_log2 = a->scale * 1.4426950408889634f;
@@ -599,8 +617,9 @@ fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const
   if (a->dtype != 0 && a->dtype != 1) return FM_ERR_UNSUPPORTED;
   if (a->D != 64 && a->D != 128) return FM_ERR_UNSUPPORTED;
   if (a->dtype == 1 && a->D != 64) return FM_ERR_UNSUPPORTED;  // fp32 tiles of D=128 exceed shared memory
-  if (a->n_q % kTile || a->n_k % kTile) return FM_ERR_UNSUPPORTED;
-  if (a->n_k / kTile > kMaxList || a->n_q / kTile > kMaxList) return FM_ERR_UNSUPPORTED;  // lists held in smem
+  if (a->n_k % 4) return FM_ERR_UNSUPPORTED;  // key tiles' bound vectors are staged by 16-byte bulk copies
+  if ((a->n_k + kTile - 1) / kTile > kMaxList || (a->n_q + kTile - 1) / kTile > kMaxList)
+    return FM_ERR_UNSUPPORTED;  // lists held in smem
   if (!a->q || !a->k || !a->v) return FM_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->k) | reinterpret_cast<uintptr_t>(a->v)) & 15)
     return FM_ERR_INVALID_ARG;

@@ -103,7 +103,7 @@ def _attn(L, n_q=256, n_k=256, D=128, dtype=0, meta_nq=None, Hm=1, H=2):
 def test_fwd_rejects_before_launch(L):
     vec = fm.VecArray(None, None, None, None)
     o, lse = ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000)
-    a, m = _attn(L, n_q=200)
+    a, m = _attn(L, n_k=202)  # key length not a multiple of 4 (ragged lengths otherwise allowed)
     assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, o, lse, None) == fm.FM_ERR_UNSUPPORTED
     a, m = _attn(L, D=96)
     assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, o, lse, None) == fm.FM_ERR_UNSUPPORTED

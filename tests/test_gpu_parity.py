@@ -282,6 +282,33 @@ def test_families_n640(fm, family):
     _compare(res, vecs, 1)
 
 
+@pytest.mark.parametrize("n,D,family", [(200, 128, "causal_document"), (388, 64, "share_question"), (4, 128, "full"),
+                                         (1000, 128, "sliding_window_2k"), (132, 128, "random_eviction"),
+                                         (676, 64, "prefix_lm_document")])
+def test_ragged_lengths(fm, n, D, family):
+    """Lengths that are not multiples of 128: zero-filled tail rows of the last tiles, the last key
+    tile always interval-tested, padded backward rows; every real row and column compared."""
+    vecs = _vec_stack(synth.make_family(family, n, 61), 1, 1)
+    res = _run_attention(fm, 1, 2, n, n, D, vecs, 1, seed=62)
+    _compare(res, vecs, 1)
+
+
+def test_ragged_cross_lengths(fm):
+    n_q, n_k = 77, 516
+    r = np.random.default_rng(63)
+    vecs = [r.integers(-10, n_q + 10, n_k).astype(np.int32)[None, None] for _ in range(4)]
+    res = _run_attention(fm, 2, 2, n_q, n_k, 128, [np.broadcast_to(v, (2, 1, n_k)).copy() for v in vecs], 1,
+                         seed=64)
+    _compare(res, [np.broadcast_to(v, (2, 1, n_k)).copy() for v in vecs], 1)
+
+
+def test_ragged_fp32(fm):
+    n = 200
+    docs = synth.cut_segments(synth.Rng(65), n, 3)
+    vecs = _vec_stack(synth.mask_causal_document(n, docs), 1, 1)
+    _compare(_run_fp32(fm, 1, 2, n, vecs, 66), vecs, 1)
+
+
 def test_dead_rows_and_cross_lengths(fm):
     n_q, n_k = 256, 512
     r = np.random.default_rng(3)

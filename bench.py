@@ -102,25 +102,64 @@ def unmasked_pairs(spec_rows, n):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and clock-event reasons of this process's GPU during the timed region, read (never
+    set) through NVML every ~5 ms from a thread; the device is found by its PCI bus id.  Falls back
+    to an `nvidia-smi -lms 200` stream when NVML is unavailable."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, dev_index):
         self.dev = dev_index
-        self.proc = None
+        self.proc = self.thread = None
+        self.samples, self.lines, self.max_mhz = [], [], None
+
+    def _nvml_start(self):
+        import threading
+
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(self.dev)
+        bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        bits = [pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap]
+        self.stop = threading.Event()
+
+        def run():
+            while True:
+                try:
+                    mhz = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((mhz, [n for n, bit in zip(self.NAMES, bits) if rs & bit]))
+                except Exception:
+                    pass
+                if self.stop.wait(0.005):
+                    break
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._nvml_start()
         except Exception:
-            self.proc = None
+            self.thread = None
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self.proc = None
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -128,28 +167,25 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
                 out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            for ln in out.splitlines():
+                f = [x.strip() for x in ln.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    self.samples.append((float(f[1]), [n for k, n in enumerate(self.NAMES)
+                                                       if f[5 + k].lower().startswith("active")]))
+                    self.max_mhz = float(f[2])
+                except ValueError:
+                    continue
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for k, name in enumerate(names):
-                if f[5 + k].lower().startswith("active"):
-                    reasons.add(name)
+        sm = [x for x, _ in self.samples]
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"]}
-        load = [x for x in sm if x > 0.5 * (mx or max(sm))] or sm
-        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        load = [x for x in sm if x > 0.5 * (self.max_mhz or max(sm))] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(sm), "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 def peaks():
@@ -279,43 +315,42 @@ def run_ours(args, rank, world, local_rank):
 
     n_loc = [sum(x) for x in loc_lens]
     nm = len(wl["masks"])
-    last = {"meta": [None] * nm}
-    state = {}
 
-    # The step as an ordered list of phases (kind, callable, kernel launches): localization of the
-    # simulated ranks, their KV-chunk pair counts, then metadata, forward and backward per mask.
-    def p_loc():
-        state["loc"] = fm.fm_localize([vec_dev[0][c] for c in range(4)], loc_starts, loc_lens)
+    def build_phases(bs):
+        """The step over one buffer set, as an ordered list of phases (kind, callable, kernel
+        launches): localization of the simulated ranks, their KV-chunk pair counts, then metadata,
+        forward and backward per mask."""
+        bs["last"], bs["state"] = {"meta": [None] * nm}, {}
+        last, state, vd = bs["last"], bs["state"], bs["vec"]
 
-    def p_kv():
-        last["pairs"] = fm.fm_kv_chunk_pairs(state["loc"], n_loc, chunk)
+        def p_loc():
+            state["loc"] = fm.fm_localize([vd[0][c] for c in range(4)], loc_starts, loc_lens)
 
-    phases = [("localize", p_loc, 1), ("kv_chunk_pairs", p_kv, 1)]
-    for mi in range(nm):
-        def p_meta(mi=mi):
-            last["meta"][mi] = fm.fm_build_mask_meta(*vec_dev[mi], n_q=n)
+        def p_kv():
+            last["pairs"] = fm.fm_kv_chunk_pairs(state["loc"], n_loc, chunk)
 
-        def p_fwd(mi=mi):
-            fm.fm_attn_fwd(q, k, v, last["meta"][mi], vec_dev[mi], scale, o=o, lse=lse)
+        ph = [("localize", p_loc, 1), ("kv_chunk_pairs", p_kv, 1)]
+        for mi in range(nm):
+            def p_meta(mi=mi):
+                last["meta"][mi] = fm.fm_build_mask_meta(*vd[mi], n_q=n)
 
-        def p_bwd(mi=mi):
-            fm.fm_attn_bwd(q, k, v, o, lse, do, last["meta"][mi], vec_dev[mi], scale, dq=dq, dk=dk, dv=dv, ws=bws)
-        phases += [("meta", p_meta, 3), ("fwd", p_fwd, 1), ("bwd", p_bwd, 3)]
-    launches_per_step = sum(x[2] for x in phases)
+            def p_fwd(mi=mi):
+                fm.fm_attn_fwd(bs["q"], bs["k"], bs["v"], last["meta"][mi], vd[mi], scale, o=bs["o"], lse=bs["lse"])
 
-    import torch.distributed as dist
-    for _ in range(args.warmup):
-        for _, fn, _ in phases:
-            fn()
-    torch.cuda.synchronize()
-    # Each phase is captured in its own CUDA graph (the host cost of the ctypes calls and output
-    # allocations would otherwise leave the GPU idle between the small kernels); events between
-    # the graph launches time the phases.
-    runners, graphs_used = [fn for _, fn, _ in phases], False
-    if not args.no_graph:
+            def p_bwd(mi=mi):
+                fm.fm_attn_bwd(bs["q"], bs["k"], bs["v"], bs["o"], bs["lse"], bs["do"], last["meta"][mi], vd[mi], scale,
+                               dq=bs["dq"], dk=bs["dk"], dv=bs["dv"], ws=bws)
+            ph += [("meta", p_meta, 3), ("fwd", p_fwd, 1), ("bwd", p_bwd, 3)]
+        return ph
+
+    def capture(ph):
+        """Each phase in its own CUDA graph (the host cost of the ctypes calls and output allocations
+        would otherwise leave the GPU idle between the small kernels); eager launches if capture fails."""
+        if args.no_graph:
+            return [fn for _, fn, _ in ph], False
         try:
             graphs = []
-            for _, fn, _ in phases:
+            for _, fn, _ in ph:
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
                     fn()
@@ -323,9 +358,22 @@ def run_ours(args, rank, world, local_rank):
             for g in graphs:  # one replay of the whole step before timing
                 g.replay()
             torch.cuda.synchronize()
-            runners, graphs_used = [g.replay for g in graphs], True
+            return [g.replay for g in graphs], True
         except Exception as exc:  # keep the eager launches (same kernels)
             print(f"bench: graph capture failed ({exc}); timing eager launches", file=sys.stderr)
+            return [fn for _, fn, _ in ph], False
+
+    bufs = [dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, vec=vec_dev)]
+    phases = build_phases(bufs[0])
+    last = bufs[0]["last"]
+    launches_per_step = sum(x[2] for x in phases)
+
+    import torch.distributed as dist
+    for _ in range(args.warmup):
+        for _, fn, _ in phases:
+            fn()
+    torch.cuda.synchronize()
+    runners, graphs_used = capture(phases)
     if world > 1:
         dist.barrier()
 
@@ -358,40 +406,79 @@ def run_ours(args, rank, world, local_rank):
     steps = args.steps
     value = job_tflops(world, flops_fwd + flops_bwd, steps, total_ms)
 
-    # end-to-end through the public API with host buffers (H2D of inputs, D2H of results)
+    # End to end through the public API with host buffers: every step copies its inputs host -> device
+    # from pinned memory and its results device -> host.  Two buffer sets are pipelined: the inputs of
+    # step s+1 go up on one copy stream and the results of step s-1 come back on another while step s
+    # computes; events order every reuse of a buffer set.
     e2e = None
     if not args.no_e2e:
-        out_host = {x: torch.empty_like(host["q"] if x in ("o", "dq") else host["k"]).pin_memory()
-                    for x in ("o", "dq", "dk", "dv")}
-        lse_host = torch.empty((B, H, n), dtype=torch.float32).pin_memory()
+        bufs.append({x: torch.empty_like(bufs[0][x]) for x in ("q", "k", "v", "do", "o", "lse", "dq", "dk", "dv")})
+        bufs[1]["vec"] = [[torch.empty_like(t) for t in vs] for vs in vec_dev]
+        run_e2e = [runners, capture(build_phases(bufs[1]))[0]]
+        out_host = [{x: torch.empty_like(bufs[0][x], device="cpu").pin_memory() for x in ("o", "dq", "dk", "dv", "lse")}
+                    for _ in range(2)]
         h2d = sum(host[x].numel() * 2 for x in host) + sum(t_.numel() * 4 for vs in vec_host for t_ in vs)
         d2h = 4 * q.numel() * 2 + lse.numel() * 4
+        up, down = torch.cuda.Stream(), torch.cuda.Stream()
+        new_ev = torch.cuda.Event
+        inputs_ready = [new_ev(), new_ev()]
+        compute_done = [new_ev(), new_ev()]
+        outputs_read = [new_ev(), new_ev()]
 
-        def e2e_step():
-            for x, dst in (("q", q), ("k", k), ("v", v), ("do", do)):
-                dst.copy_(host[x], non_blocking=True)
-            for mi, vs in enumerate(vec_host):
-                for c in range(4):
-                    vec_dev[mi][c].copy_(vs[c], non_blocking=True)
-            step()
-            for x, src in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
-                out_host[x].copy_(src, non_blocking=True)
-            lse_host.copy_(lse, non_blocking=True)
+        def upload(s_):  # inputs of step s_ into buffer set s_ % 2
+            bs = bufs[s_ % 2]
+            with torch.cuda.stream(up):
+                if s_ >= 2:
+                    up.wait_event(compute_done[s_ % 2])  # step s_-2 has finished reading this set
+                for x in ("q", "k", "v", "do"):
+                    bs[x].copy_(host[x], non_blocking=True)
+                for mi, vs in enumerate(vec_host):
+                    for c in range(4):
+                        bs["vec"][mi][c].copy_(vs[c], non_blocking=True)
+                inputs_ready[s_ % 2].record(up)
 
-        for _ in range(max(1, args.warmup // 2)):
-            e2e_step()
-        torch.cuda.synchronize()
+        def compute(s_):
+            stream.wait_event(inputs_ready[s_ % 2])
+            if s_ >= 2:
+                stream.wait_event(outputs_read[s_ % 2])  # results of step s_-2 are home
+            for run in run_e2e[s_ % 2]:
+                run()
+            compute_done[s_ % 2].record(stream)
+
+        def download(s_):
+            bs, oh = bufs[s_ % 2], out_host[s_ % 2]
+            with torch.cuda.stream(down):
+                down.wait_event(compute_done[s_ % 2])
+                for x in ("o", "dq", "dk", "dv", "lse"):
+                    oh[x].copy_(bs[x], non_blocking=True)
+                outputs_read[s_ % 2].record(down)
+
+        def pipeline(nsteps, e_start=None, e_end=None):
+            torch.cuda.synchronize()
+            if e_start is not None:
+                e_start.record(stream)
+                up.wait_event(e_start)
+                down.wait_event(e_start)
+            upload(0)
+            for s_ in range(nsteps):
+                if s_ + 1 < nsteps:
+                    upload(s_ + 1)
+                compute(s_)
+                download(s_)
+            stream.wait_event(outputs_read[(nsteps - 1) % 2])
+            if e_end is not None:
+                e_end.record(stream)
+            torch.cuda.synchronize()
+
+        pipeline(max(2, args.warmup))
         if world > 1:
             dist.barrier()
         e0, e1 = ev(), ev()
-        e0.record(stream)
-        for _ in range(steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        pipeline(steps, e0, e1)
         (te_ms,) = reduce_max([e0.elapsed_time(e1)], world, dev)
         e2e = {"value": job_tflops(world, flops_fwd + flops_bwd, steps, te_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "note": "inputs of step s+1 uploaded and results of step s-1 downloaded while step s computes"}
     assert fm.fm_get_device_status() == 0, "device-side timeout during the bench"
 
     burst, sustained, hbm, src = peaks()

@@ -177,6 +177,23 @@ def test_kv_chunk_pairs_bitexact(fm):
         np.testing.assert_array_equal(nul[rr, 0, 0], oracle.kv_chunk_pairs(n_loc[rr], N, chunk, None, None, None, lv))
 
 
+def test_chunk_costs_and_balanced_assignment(fm):
+    """Per-query-chunk work measured by the GPU passes equals the oracle's counts; the
+    longest-first assignment balances a document mask at least as well as dual-chunk."""
+    from mask_aware_flash_b200 import cp_balance as cb
+    N, chunk = 8192, 256
+    spec = synth.mask_causal_document(N, synth.draw_docs(synth.Rng(71), N, 256, 2048))
+    vt = [torch.from_numpy(np.ascontiguousarray(x[None, None])).cuda() for x in spec.vectors()]
+    cost = cb.chunk_costs(fm, vt, chunk)
+    want = []
+    for c in range(N // chunk):
+        loc = [oracle.localize(x, [c * chunk], [chunk]) for x in spec.vectors()]
+        want.append(int(oracle.kv_chunk_pairs(chunk, N, N, *loc).sum()))
+    np.testing.assert_array_equal(cost, want)
+    assert cb.imbalance(cost, cb.assign_longest_first(cost, N // chunk // 2, 2)) <= \
+        cb.imbalance(cost, cb.dual_chunk(N // chunk)) + 1e-12
+
+
 # ---------------------------------------------------------------------------- attention
 def _run_attention(fm, B, H, n_q, n_k, D, vecs_np, Hm, seed, scale=None, bwd=True):
     scale = 1.0 / math.sqrt(D) if scale is None else scale

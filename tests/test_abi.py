@@ -105,6 +105,10 @@ def test_fwd_rejects_before_launch(L):
     o, lse = ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000)
     a, m = _attn(L, n_k=202)  # key length not a multiple of 4 (ragged lengths otherwise allowed)
     assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, o, lse, None) == fm.FM_ERR_UNSUPPORTED
+    a, m = _attn(L, n_q=4097 * 128)  # one query tile more than the lists hold
+    assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, o, lse, None) == fm.FM_ERR_UNSUPPORTED
+    a, m = _attn(L, n_k=4097 * 128)
+    assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, o, lse, None) == fm.FM_ERR_UNSUPPORTED
     a, m = _attn(L, D=96)
     assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, o, lse, None) == fm.FM_ERR_UNSUPPORTED
     a, m = _attn(L, dtype=1)

@@ -193,3 +193,28 @@ def test_localization_262144_16_ranks(fm):
         ref = oracle.attention_head(*host[:3], vecs, 0, h, scale, rows=rows)
         _check_rows(go, glse, None, ref, 0, h)
     assert fm.fm_get_device_status() == 0
+
+
+def test_maximum_tile_count_524288(fm):
+    """The largest length the row / column lists hold: 4096 tiles of 128 (n = 524288).  Global +
+    sliding window (128 global tokens, band 512): query tile 0 sees every key tile and key tile 0 is
+    seen by every query tile, so both a row list and a column list hold all 4096 entries, while the
+    oracle's all-rows pass stays affordable.  Sampled rows (O, LSE, dQ) and sampled columns (dK, dV)
+    against the oracle; one tile more is rejected on the host (test_abi)."""
+    n, B, H, D = 524288, 1, 1, 128
+    host, dev = _inputs(B, n, H, D, 7000)
+    spec = synth.mask_global_sliding(n, 128, 512)
+    vecs = [x[None, None] for x in spec.vectors()]
+    scale = 1.0 / math.sqrt(D)
+    vt = [torch.from_numpy(np.ascontiguousarray(v)).cuda() for v in vecs]
+    meta = fm.fm_build_mask_meta(*vt, n_q=n)
+    o, lse = fm.fm_attn_fwd(dev[0], dev[1], dev[2], meta, vt, scale)
+    dq, dk, dv = fm.fm_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], meta, vt, scale)
+    torch.cuda.synchronize()
+    assert fm.fm_get_device_status() == 0
+    assert int(meta.row_count[0, 0, 0].item()) == 4096 and int(meta.col_count[0, 0, 0].item()) == 4096
+    rows = _sample(n, N_SAMPLE, 7001, extra=[0, 127, 128, n - 129, n - 1])
+    cols = _sample(n, N_SAMPLE, 7002, extra=[0, 127, 128, n - 1])
+    ref = oracle.attention_head(*host[:3], vecs, 0, 0, scale, rows=rows, cols=cols, dout=host[3])
+    _check_rows(o, lse, dq, ref, 0, 0)
+    _check_cols(dk, dv, ref, 0, 0)

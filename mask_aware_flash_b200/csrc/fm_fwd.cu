@@ -36,7 +36,7 @@ constexpr int kFwdThreads = 320;
 constexpr int kMaxList = 4096;  // key tiles per query tile held in shared memory (n_k <= 524288)
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
-constexpr int kPolyEvery = 4;  // one score pair in kPolyEvery takes exp2_poly2 instead of MUFU ex2
+constexpr int kPolyEvery = 8;  // one score pair in kPolyEvery takes exp2_poly2 instead of MUFU ex2
 constexpr float kLiveSum = 1e-20f;  // a live row's sum is >= ~1; masked scores add ~2^-125 each
 
 struct FwdParams {

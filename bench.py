@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the phases eagerly instead of graph replays")
+    ap.add_argument("--no-aux", action="store_true", help="skip the batched integer-pass measurement")
     return ap.parse_args()
 
 
@@ -505,7 +506,7 @@ def run_ours(args, rank, world, local_rank):
         "kv_chunk_pairs": dict(bw(16 * B * n * R + 8 * pairs.numel(), kvc_ms, steps), ranks=R,
                                chunks_pruned=int((pairs == 0).sum().item()), chunks=int(pairs.numel()),
                                rank_work_max_over_mean=round(float(rank_work.max() / rank_work.mean()), 4)),
-        "batched_n262144_r16": aux_localize(fm, torch, dev, stream, hbm),
+        "batched_n262144_r16": None if args.no_aux else aux_localize(fm, torch, dev, stream, hbm),
     }
     fwd_tf = flops_fwd * steps / (fwd_ms * 1e-3) / 1e12
     bwd_tf = flops_bwd * steps / (bwd_ms * 1e-3) / 1e12

@@ -24,7 +24,8 @@
  *     Any int32 value is legal; start >= end is an empty stretch.  A NULL vector
  *     pointer stands for its canonical empty value (LTS = LTE = n_q, UTS = UTE = 0).
  *     Vectors are int32 [B, Hm, n_k] contiguous, Hm = 1 (shared by all heads) or H.
- *   - Tensors Q, O, dO, dQ are [B, n_q, H, D] and K, V, dK, dV are [B, n_k, H, D],
+ *   - Tensors Q, O, dO, dQ are [B, n_q, H, D] and K, V, dK, dV are [B, n_k, H_kv, D] (H_kv = H
+ *     unless fm_attn_args.H_kv says otherwise: grouped-query attention),
  *     contiguous, all of one element type: bf16 (dtype 0; bf16 tensor-core products) or
  *     fp32 (dtype 1, D = 64 only; tf32 tensor-core products, fp32 accumulation).  LSE is
  *     fp32 [B, H, n_q], natural log.
@@ -171,6 +172,8 @@ typedef struct {
   const void* q;
   const void* k;
   const void* v;
+  int32_t H_kv;   /* K/V heads (grouped-query attention): H % H_kv == 0, query head h reads K/V
+                     head h / (H / H_kv); 0 means H_kv = H */
 } fm_attn_args;
 
 /*
@@ -179,7 +182,8 @@ typedef struct {
  * LSE_i = ln sum_{j in U_i} exp(scale q_i.k_j); a row with U_i empty gets
  * O_i = 0 and LSE_i = -inf.  Only non-skip key tiles (meta row lists) are read;
  * the row-interval test runs on partial tiles only.
- *   a      host struct; n_q >= 1 any length, n_k >= 1 a multiple of 4 (ragged lengths: the last
+ *   a      host struct; H_kv divides H (0 = H; at most 64 query heads per K/V head);
+ *          n_q >= 1 any length, n_k >= 1 a multiple of 4 (ragged lengths: the last
  *          tiles are zero-filled past n and the last key tile always runs the interval test);
  *          at most 4096 tiles each way; D in {64, 128}; dtype 0, or 1 with D = 64;
  *          scale > 0 and finite.
@@ -202,7 +206,10 @@ size_t fm_attn_bwd_workspace_bytes(const fm_attn_args* a);
  *   dQ_i = scale sum_j dS_ij k_j, dK_j = scale sum_i dS_ij q_i.
  * Key tiles iterate their meta column lists (non-skip query tiles only).
  *   o, lse   the forward's outputs; dout device [B, n_q, H, D] of the dtype.
- *   dq, dk, dv device outputs of the dtype (layouts above); every element is written.
+ *   dq, dk, dv device outputs of the dtype; dq [B, n_q, H, D], dk / dv [B, n_k, H_kv, D] (the
+ *            gradient of a shared K/V head sums over its query heads); every element is written.
+ *   The column lists of the query heads sharing a K/V head are held together: (H / H_kv) x
+ *   ceil(n_q / 128) <= 4096, else FM_ERR_UNSUPPORTED.
  *   ws       device workspace, ws_bytes >= fm_attn_bwd_workspace_bytes(a), 256-byte
  *            aligned; holds the fp32 dQ accumulator and per-row statistics.
  * Errors: FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA.

@@ -49,7 +49,7 @@ class MaskMetaC(ctypes.Structure):
 class AttnArgs(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("n_q", ctypes.c_int32), ("n_k", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p)]
+                ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("H_kv", ctypes.c_int32)]
 
 
 VecArray = ctypes.c_void_p * 4
@@ -195,12 +195,13 @@ def fm_kv_chunk_pairs(loc_vecs, n_loc, chunk_len: int, out=None, stream=None):
 def _args(q, k, v, scale) -> AttnArgs:
     B, n_q, H, D = q.shape
     dtype = 1 if q.dtype == torch.float32 else 0
-    return AttnArgs(B, H, n_q, k.shape[1], D, dtype, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr())
+    return AttnArgs(B, H, n_q, k.shape[1], D, dtype, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                    k.shape[2])
 
 
 def fm_attn_fwd(q, k, v, meta: MaskMeta, vecs, scale, o=None, lse=None, stream=None):
-    """q [B, n_q, H, D], k/v [B, n_k, H, D] CUDA tensors (bf16, or fp32 with D=64) -> o (same dtype),
-    lse [B, H, n_q] fp32."""
+    """q [B, n_q, H, D], k/v [B, n_k, H_kv, D] CUDA tensors (bf16, or fp32 with D=64; H % H_kv == 0)
+    -> o (same dtype), lse [B, H, n_q] fp32."""
     B, n_q, H, D = q.shape
     if o is None:
         o = torch.empty_like(q)
@@ -224,7 +225,7 @@ def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=No
     nbytes = lib().fm_attn_bwd_workspace_bytes(ctypes.byref(a))
     if ws is None:
         ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    dq = torch.empty_like(q) if dq is None else dq
+    dq = torch.empty_like(q) if dq is None else dq  # dk, dv: the shape of k, v ([B, n_k, H_kv, D])
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     _check(lib().fm_attn_bwd(ctypes.byref(a), ctypes.byref(meta.c), _vecs(vecs), _ptr(o), _ptr(lse), _ptr(do),

@@ -48,6 +48,7 @@ struct BwdParams {
   int* status;
   int B, H, Hm, n_q, n_k, T_q, T_k;
   int n_q_pad;                 // n_q rounded up to whole query tiles (row stride of lse2, dvec, dq_acc)
+  int H_kv, q_per_kv;          // K/V heads; query heads per K/V head (grouped-query attention)
   int group;                   // heads dispatched together
   float scale, scale_log2;
 };
@@ -70,7 +71,8 @@ struct BwdSmem {
   static constexpr int kDS = kDO + kQStages * kQStage;  // kDSBufs buffers
   static constexpr int kStats = kDS + kDSBufs * kDSBytes;  // kQStages x (64 lse2 + 64 D_i) fp32
   static constexpr int kList = kStats + kQStages * 2 * kBQ * 4;  // column list, uint16
-  static constexpr int kBar = kList + kMaxList * 2;
+  static constexpr int kHeads = kList + kMaxList * 2;  // [q_per_kv + 1] list offsets, int32 (<= 65)
+  static constexpr int kBar = kHeads + 65 * 4 + 12;      // (8-byte aligned)
   enum { KV_FULL, QDO_FULL0, QDO_FULL1, QDO_FULL2, QDO_EMPTY0, QDO_EMPTY1, QDO_EMPTY2, SDP_FULL, DP_FREE,
          DS_READY, DS_EMPTY0, DS_EMPTY1, DQ_FULL, DQ_EMPTY, ACC_FULL, DRAIN,
          QT_GO0, QT_GO1, QT_READY0, QT_READY1, KT_READY,  // fp32 path: operand transposes
@@ -138,14 +140,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // grid (group * T_k, ceil(H / group), B): a group of heads at a time, rank by rank over the
   // group's heads (rank r takes the key tile with the r-th longest column list); the group is sized
   // so that its heads' Q, dO and dQ accumulator stay in L2
-  const int h = (int)blockIdx.y * p.group + (int)(blockIdx.x % p.group), b = blockIdx.z;
-  if (h >= p.H) return;  // partial last group
-  const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
-  const int kt = __ldg(p.order + bhm * p.T_k + blockIdx.x / p.group);
-  const int64_t bh = (int64_t)b * p.H + h;
-  const int cnt = __ldg(p.col_count + bhm * p.T_k + kt);
+  // One CTA per (key tile, K/V head hk).  With grouped-query attention the q_per_kv query heads
+  // hk * q_per_kv + j share this K/V head: their column lists are walked back to back (dK and dV
+  // accumulate over all of them); the list of head j starts at entry hstart[j].
+  const int hk = (int)blockIdx.y * p.group + (int)(blockIdx.x % p.group), b = blockIdx.z;
+  if (hk >= p.H_kv) return;  // partial last group
+  const int G = p.q_per_kv, hq0 = hk * G;
+  auto bhm_of = [&](int hq) -> int64_t { return (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : hq); };
+  const int kt = __ldg(p.order + bhm_of(hq0) * p.T_k + blockIdx.x / p.group);
+  int cnt = 0;  // entries over the group's query heads
+  for (int jq = 0; jq < G; ++jq) cnt += __ldg(p.col_count + bhm_of(hq0 + jq) * p.T_k + kt);
   const int nsub = 2 * cnt;  // two 64-row sub-tiles per listed 128-row query tile
-  const int32_t* entries = p.col_entries + (bhm * p.T_k + kt) * p.T_q;
 
   const uint32_t bar0 = smem_u32(smem + S::kBar);
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -174,12 +179,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&tm_v);
       mbar_arrive_expect_tx(bar(S::KV_FULL), 2 * kTile * D * S::kElem);
       for (int c = 0; c < kAtoms; ++c) {
-        tma_load_4d(k_s + c * 16384, &tm_k, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
-        tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * kAtomElems, h, kt * kTile, b);
+        tma_load_4d(k_s + c * 16384, &tm_k, bar(S::KV_FULL), c * kAtomElems, hk, kt * kTile, b);
+        tma_load_4d(v_s + c * 16384, &tm_v, bar(S::KV_FULL), c * kAtomElems, hk, kt * kTile, b);
       }
     }
   }
-  for (int t = threadIdx.x; t < cnt; t += kBwdThreads) list[t] = (uint16_t)__ldg(entries + t);
+  int* hstart = reinterpret_cast<int*>(smem + S::kHeads);  // [G + 1]
+  {
+    int start = 0;
+    for (int jq = 0; jq < G; ++jq) {
+      const int64_t bj = bhm_of(hq0 + jq);
+      const int cj = __ldg(p.col_count + bj * p.T_k + kt);
+      const int32_t* ej = p.col_entries + (bj * p.T_k + kt) * p.T_q;
+      if (threadIdx.x == 0) hstart[jq] = start;
+      for (int t = threadIdx.x; t < cj; t += kBwdThreads) list[start + t] = (uint16_t)__ldg(ej + t);
+      start += cj;
+    }
+    if (threadIdx.x == 0) hstart[G] = start;
+  }
   if (!F32 && kAtoms * 128 * kTile < S::kKBytes) {  // K^T as a 128-row MMA operand: rows d >= D read zeros
     uint4* z = reinterpret_cast<uint4*>(smem + S::kK + kAtoms * 128 * kTile);
     for (int t = threadIdx.x; t < (S::kKBytes - kAtoms * 128 * kTile) / 16; t += blockDim.x)
@@ -198,12 +215,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // fp32 (D = 64): dS^T [320,384) as the TMEM operand of dK
   const uint32_t tdP = tmem + 128, tdQ = tmem + 192, tdV = tmem + 256, tdK = tmem + 384, tdS = tmem + 320;
   auto sub_q0 = [&](int i) { return (int)(list[i >> 1] >> 1) * kTile + (i & 1) * kBQ; };
+  // query head (offset in the group) of sub-tile i; each role advances its own cursor jh
+  auto head_of = [&](int i, int& jh) {
+    while ((i >> 1) >= hstart[jh + 1]) ++jh;
+    return jh;
+  };
 
   if (warp == 12) {
     // ------------------------------------------------------------ load role
     if (lane == 0 && cnt > 0) {
       prefetch_tmap(&tm_q);  // (K and V were issued at the start)
       prefetch_tmap(&tm_do);
+      int jh = 0;
       for (int i = 0; i < nsub; ++i) {
         const int st = i % NS, use = i / NS;
         if (use >= 1 && !mbar_wait(bar(S::QDO_EMPTY0 + st), (use - 1) & 1, abort_flag)) {
@@ -211,11 +234,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         const int q0 = sub_q0(i);
+        const int hq = hq0 + head_of(i, jh);
+        const int64_t bh = (int64_t)b * p.H + hq;
         const uint32_t fb = bar(S::QDO_FULL0 + st);
         mbar_arrive_expect_tx(fb, 2 * S::kQStage + 2 * kBQ * 4);
         for (int c = 0; c < kAtoms; ++c) {
-          tma_load_4d(q_s + st * S::kQStage + c * 8192, &tm_q, fb, c * kAtomElems, h, q0, b);
-          tma_load_4d(do_s + st * S::kQStage + c * 8192, &tm_do, fb, c * kAtomElems, h, q0, b);
+          tma_load_4d(q_s + st * S::kQStage + c * 8192, &tm_q, fb, c * kAtomElems, hq, q0, b);
+          tma_load_4d(do_s + st * S::kQStage + c * 8192, &tm_do, fb, c * kAtomElems, hq, q0, b);
         }
         bulk_load(smem_u32(stats + st * 2 * kBQ), p.lse2 + bh * p.n_q_pad + q0, kBQ * 4, fb);
         bulk_load(smem_u32(stats + st * 2 * kBQ + kBQ), p.dvec + bh * p.n_q_pad + q0, kBQ * 4, fb);
@@ -357,14 +382,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int c0 = 32 * hf;
     const int64_t j = (int64_t)kt * kTile + r;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-    const int64_t voff = bhm * p.n_k + j;
     const bool no_key = j >= p.n_k;  // past a ragged n_k: a zero-filled key row, masked for every query
-    const int32_t lts = (p.vec[0] && !no_key) ? __ldg(p.vec[0] + voff) : p.n_q;
-    const int32_t lte = (p.vec[1] && !no_key) ? __ldg(p.vec[1] + voff) : p.n_q;
-    const int32_t uts = (p.vec[2] && !no_key) ? __ldg(p.vec[2] + voff) : 0;
-    const int32_t ute = (p.vec[3] && !no_key) ? __ldg(p.vec[3] + voff) : 0;
+    int32_t lts = p.n_q, lte = p.n_q, uts = 0, ute = 0;
+    int jh = 0, jv = -1;  // head cursor; head whose vectors are loaded
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
+      const int jq = head_of(i, jh);
+      if (jv < 0 || (p.Hm != 1 && jq != jv)) {  // this key's bounds for the sub-tile's query head
+        const int64_t voff = bhm_of(hq0 + jq) * p.n_k + j;
+        lts = (p.vec[0] && !no_key) ? __ldg(p.vec[0] + voff) : p.n_q;
+        lte = (p.vec[1] && !no_key) ? __ldg(p.vec[1] + voff) : p.n_q;
+        uts = (p.vec[2] && !no_key) ? __ldg(p.vec[2] + voff) : 0;
+        ute = (p.vec[3] && !no_key) ? __ldg(p.vec[3] + voff) : 0;
+        jv = jq;
+      }
       const int st = i % NS, bi = i % NDS, sb = i & 1;  // Q/dO stage, dS^T buffer, S^T buffer
       const int q0 = sub_q0(i) + c0;
       const bool partial = list[i >> 1] & 1;
@@ -450,7 +481,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // dP^T have read the stage)
     const int d = threadIdx.x - 256;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-    float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q_pad * D;
+    int jh = 0;
     bool ok = true;
     if constexpr (F32) {
       if (nsub > 0) {
@@ -464,6 +495,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int i = 0; ok && i < nsub; ++i) {
       const int q0 = sub_q0(i);
+      float* acc_bh = p.dq_acc + ((int64_t)b * p.H + hq0 + head_of(i, jh)) * (int64_t)p.n_q_pad * D;
       if constexpr (F32) {
         const int st = i % NS;
         ok = all_drain_threads(mbar_wait(bar(S::QT_GO0 + st), (i / NS) & 1, abort_flag));
@@ -540,7 +572,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     named_bar_sync(is_dk ? 3 : 2, 128);
     if (r == 0) {
       for (int c = 0; c < kAtoms; ++c)
-        tma_store_4d(is_dk ? &tm_dk : &tm_dv, smem_u32(stage + c * 16384), c * kAtomElems, h, kt * kTile, b);
+        tma_store_4d(is_dk ? &tm_dk : &tm_dv, smem_u32(stage + c * 16384), c * kAtomElems, hk, kt * kTile, b);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -676,11 +708,12 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   float* acc = reinterpret_cast<float*>(w + L.acc);
   float* lse2 = reinterpret_cast<float*>(w + L.lse2);
   float* dvec = reinterpret_cast<float*>(w + L.dvec);
+  const int H_kv = a->H_kv ? a->H_kv : a->H;
   CUtensorMap tq, tdo, tk, tv, tdk, tdv;
   auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
   if (!enc(&tq, a->q, D, a->H, a->n_q, a->B, kBQ) || !enc(&tdo, dout, D, a->H, a->n_q, a->B, kBQ) ||
-      !enc(&tk, a->k, D, a->H, a->n_k, a->B, kTile) || !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile) ||
-      !enc(&tdk, dk, D, a->H, a->n_k, a->B, kTile) || !enc(&tdv, dv, D, a->H, a->n_k, a->B, kTile))
+      !enc(&tk, a->k, D, H_kv, a->n_k, a->B, kTile) || !enc(&tv, a->v, D, H_kv, a->n_k, a->B, kTile) ||
+      !enc(&tdk, dk, D, H_kv, a->n_k, a->B, kTile) || !enc(&tdv, dv, D, H_kv, a->n_k, a->B, kTile))
     return FM_ERR_CUDA;
   const int64_t rows = (int64_t)a->B * a->n_q * a->H;
   bwd_prep_kernel<D, F32><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(o, dout, lse, lse2, dvec, acc, a->B,
@@ -704,17 +737,31 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.T_q = (a->n_q + kTile - 1) / kTile;
   p.T_k = (a->n_k + kTile - 1) / kTile;
   p.n_q_pad = p.T_q * kTile;
-  p.group = dispatch_group(p.H, (double)a->n_q * D * (2 * S::kElem + 4));  // Q, dO, fp32 dQ accumulator
+  p.H_kv = H_kv;
+  p.q_per_kv = a->H / H_kv;
+  // the CTAs of one K/V head re-read the Q, dO and fp32 dQ accumulator of its q_per_kv query heads
+  p.group = dispatch_group(H_kv, (double)p.q_per_kv * a->n_q * D * (2 * S::kElem + 4));
   p.scale = a->scale;
   p.scale_log2 = a->scale * 1.4426950408889634f;
   if (!smem_opt_in<bwd_kernel<D, F32>>(S::kAlloc)) return FM_ERR_CUDA;
-  bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
+  bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H_kv + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
   bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (p.n_q_pad / 64)), 256, 0, stream>>>(
       acc, dq, a->B, a->H, a->n_q, p.n_q_pad, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 
 }  // namespace
+
+// The backward's checks: the attention checks, plus room in shared memory for the column lists of
+// all query heads that share a K/V head (q_per_kv x T_q entries at most).
+fm_status check_bwd_args(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4]) {
+  const fm_status st = check_attn_args(a, meta, vec);
+  if (st != FM_OK) return st;
+  const int H_kv = a->H_kv ? a->H_kv : a->H;
+  if ((int64_t)(a->H / H_kv) * ((a->n_q + 127) / 128) > kMaxList) return FM_ERR_UNSUPPORTED;
+  return FM_OK;
+}
+
 }  // namespace fm
 
 extern "C" {
@@ -727,7 +774,7 @@ size_t fm_attn_bwd_workspace_bytes(const fm_attn_args* a) {
 fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], const void* o,
                       const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
                       fm_stream_t stream) {
-  fm_status st = fm::check_attn_args(a, meta, vec);
+  fm_status st = fm::check_bwd_args(a, meta, vec);
   if (st != FM_OK) return st;
   const uintptr_t al = reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(dout) |
                        reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
@@ -771,7 +818,7 @@ void* noalloc_scratch() {
 extern "C" fm_status fm_attn_bwd_noalloc(const fm_attn_args* a, const fm_mask_meta* meta,
                                          const int32_t* const vec[4], const void* o, const float* lse,
                                          const void* dout, void* dq, void* dk, void* dv, fm_stream_t stream) {
-  fm_status st = fm::check_attn_args(a, meta, vec);
+  fm_status st = fm::check_bwd_args(a, meta, vec);
   if (st != FM_OK) return st;
   if (fm_attn_bwd_workspace_bytes(a) > FM_BWD_NOALLOC_SCRATCH_BYTES) return FM_ERR_WORKSPACE;
   void* ws = noalloc_scratch();

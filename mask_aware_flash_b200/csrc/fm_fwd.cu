@@ -49,6 +49,7 @@ struct FwdParams {
   float* lse;                  // [B, H, n_q]
   int* status;
   int B, H, Hm, n_q, n_k, T_q, T_k, n_pairs;
+  int H_kv, q_per_kv;          // K/V heads; query heads per K/V head (grouped-query attention)
   int group;                   // heads dispatched together
   float scale_log2;            // softmax scale * log2(e), > 0
 };
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
       }
+      const int hk = h / p.q_per_kv;  // the K/V head of query head h
       int nvec = 0;
       for (int c = 0; c < 4; ++c) nvec += p.vec[c] ? 1 : 0;
       MergedList it{list0, list1, n0, n1, 0, 0, ragged_kt};
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(bar(S::K_FULL0 + slot), S::kTileBytes);
           for (int c = 0; c < kAtoms; ++c)
-            tma_load_4d(k_s + slot * S::kTileBytes + c * 16384, &tm_k, bar(S::K_FULL0 + slot), c * kAtomElems, h,
+            tma_load_4d(k_s + slot * S::kTileBytes + c * 16384, &tm_k, bar(S::K_FULL0 + slot), c * kAtomElems, hk,
                         kt * kTile, b);
         }
         if (c0 == 1 || c1 == 1) {
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         if constexpr (F32) {
           load_vt_f32<D>(smem + S::kV + slot * S::kTileBytes,
-                         p.v32 + (((int64_t)b * p.n_k + (int64_t)kt * kTile) * p.H + h) * D, (int64_t)p.H * D,
+                         p.v32 + (((int64_t)b * p.n_k + (int64_t)kt * kTile) * p.H_kv + hk) * D, (int64_t)p.H_kv * D,
                          min(kTile, p.n_k - kt * kTile), lane);
           fence_proxy_async_smem();  // generic-proxy stores, read next by the tensor core
           __syncwarp();
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         } else {
           mbar_arrive_expect_tx(bar(S::V_FULL0 + slot), S::kTileBytes);
           for (int c = 0; c < kAtoms; ++c)
-            tma_load_4d(v_s + slot * S::kTileBytes + c * 16384, &tm_v, bar(S::V_FULL0 + slot), c * kAtomElems, h,
+            tma_load_4d(v_s + slot * S::kTileBytes + c * 16384, &tm_v, bar(S::V_FULL0 + slot), c * kAtomElems, hk,
                         kt * kTile, b);
         }
         ++e;
@@ -580,8 +582,9 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   static_assert(S::kAlloc <= 227 * 1024, "forward shared memory exceeds the per-CTA limit");
   CUtensorMap tq, tk, tv, to;
   auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
-  if (!enc(&tq, a->q, D, a->H, a->n_q, a->B, kTile) || !enc(&tk, a->k, D, a->H, a->n_k, a->B, kTile) ||
-      !enc(&tv, a->v, D, a->H, a->n_k, a->B, kTile) || !enc(&to, o, D, a->H, a->n_q, a->B, kTile))
+  const int H_kv = a->H_kv ? a->H_kv : a->H;
+  if (!enc(&tq, a->q, D, a->H, a->n_q, a->B, kTile) || !enc(&tk, a->k, D, H_kv, a->n_k, a->B, kTile) ||
+      !enc(&tv, a->v, D, H_kv, a->n_k, a->B, kTile) || !enc(&to, o, D, a->H, a->n_q, a->B, kTile))
     return FM_ERR_CUDA;
   FwdParams p;
   p.row_count = meta->row_count;
@@ -594,6 +597,8 @@ fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.status = device_status_ptr();
   p.B = a->B;
   p.H = a->H;
+  p.H_kv = H_kv;
+  p.q_per_kv = a->H / H_kv;
   p.Hm = meta->d.Hm;
   p.n_q = a->n_q;
   p.n_k = a->n_k;
@@ -627,6 +632,9 @@ fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const
   if (d.B != a->B || d.n_q != a->n_q || d.n_k != a->n_k || d.tile_q != kTile || d.tile_k != kTile)
     return FM_ERR_INVALID_ARG;
   if (d.Hm != 1 && d.Hm != a->H) return FM_ERR_INVALID_ARG;
+  const int H_kv = a->H_kv ? a->H_kv : a->H;  // grouped-query attention: H_kv divides H
+  if (H_kv < 1 || H_kv > a->H || a->H % H_kv) return FM_ERR_INVALID_ARG;
+  if (a->H / H_kv > 64) return FM_ERR_UNSUPPORTED;  // the backward's per-CTA head table
   if (!meta->row_count || !meta->row_entries || !meta->col_count || !meta->col_entries || !meta->fwd_order ||
       !meta->bwd_order)
     return FM_ERR_INVALID_ARG;

@@ -326,6 +326,50 @@ def test_ragged_fp32(fm):
     _compare(_run_fp32(fm, 1, 2, n, vecs, 66), vecs, 1)
 
 
+@pytest.mark.parametrize("H,H_kv,Hm,D", [(4, 2, 1, 128), (4, 1, 1, 64), (6, 2, 6, 128), (8, 8, 1, 64)])
+def test_grouped_query_heads(fm, H, H_kv, Hm, D):
+    """Grouped-query attention: K / V have H_kv heads, query head h reads K/V head h // (H / H_kv).
+    The oracle sees K / V repeated to H heads; the reference dK / dV of a K/V head is the sum over
+    its query heads of their gradients (the plain chain rule through the repetition)."""
+    n, seed, g = 640, 81, H // H_kv
+    fams = ["causal_document", "share_question", "sliding_window_2k", "prefix_lm", "random_eviction", "full"]
+    if Hm == 1:
+        vecs = _vec_stack(synth.make_family("causal_document", n, seed), 1, 1)
+    else:
+        specs = [synth.make_family(fams[h % len(fams)], n, seed + h) for h in range(H)]
+        vecs = [np.stack([sp.vectors()[c] for sp in specs])[None] for c in range(4)]  # [1, H, n]
+    bits = [synth.normal_bf16_bits(seed, t, (1, n, hh, D)) for t, hh in ((1, H), (2, H_kv), (3, H_kv), (4, H))]
+    host = [synth.bf16_bits_to_f32(x) for x in bits]
+    dev = [_bf16_tensor(x) for x in bits]
+    vt = [torch.from_numpy(np.ascontiguousarray(v, np.int32)).cuda() for v in vecs]
+    scale = 1.0 / math.sqrt(D)
+    meta = fm.fm_build_mask_meta(*vt, n_q=n)
+    o, lse = fm.fm_attn_fwd(dev[0], dev[1], dev[2], meta, vt, scale)
+    dq, dk, dv = fm.fm_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], meta, vt, scale)
+    torch.cuda.synchronize()
+    assert fm.fm_get_device_status() == 0
+    assert dk.shape == (1, n, H_kv, D)
+    k_exp, v_exp = np.repeat(host[1], g, axis=2), np.repeat(host[2], g, axis=2)
+    dk_ref = np.zeros((n, H_kv, D))
+    dv_ref = np.zeros((n, H_kv, D))
+    o_np, lse_np, dq_np = o.float().cpu().numpy(), lse.cpu().numpy(), dq.float().cpu().numpy()
+    for h in range(H):
+        ref = oracle.attention_head(host[0], k_exp, v_exp, vecs, 0, h, scale, cols=np.arange(n), dout=host[3],
+                                    Hm=Hm)
+        live = np.isfinite(ref["lse"])
+        assert np.abs(o_np[0, :, h] - ref["o"]).max() <= O_TOL
+        if live.any():
+            assert np.abs(lse_np[0, h][live] - ref["lse"][live]).max() <= LSE_TOL
+        assert np.abs(dq_np[0, :, h] - ref["dq"]).max() <= G_TOL * max(np.abs(ref["dq"]).max(), 1e-30)
+        dk_ref[:, h // g] += ref["dk"]
+        dv_ref[:, h // g] += ref["dv"]
+    for name, got, exp in (("dk", dk, dk_ref), ("dv", dv, dv_ref)):
+        for hk in range(H_kv):
+            e = exp[:, hk]
+            err = np.abs(got.float().cpu().numpy()[0, :, hk] - e).max() / max(np.abs(e).max(), 1e-30)
+            assert err <= G_TOL, f"{name} head {hk}: rel-to-max {err}"
+
+
 def test_dead_rows_and_cross_lengths(fm):
     n_q, n_k = 256, 512
     r = np.random.default_rng(3)

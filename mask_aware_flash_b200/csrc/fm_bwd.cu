@@ -7,18 +7,21 @@
 // tile walks its column list of non-skip query tiles and applies the
 // row-interval test only on partial tiles.
 //
-// Per key tile of 128 keys (one CTA), per 64-row query sub-tile:
+// Per key tile of 128 keys (one CTA; with grouped-query attention, per key
+// tile and K/V head), per 64-row query sub-tile of its column list:
 //   S^T  = K Q^T        (tcgen05, M=128 keys, N=64 queries)      -> TMEM
 //   dP^T = V dO^T       (tcgen05)                                -> TMEM
-//   P^T  = 2^(S^T scale log2e - LSE2), masked entries 0         (warps 0-3)
-//   dS^T = P^T (dP^T - D_i)                                     (warps 0-3)
+//   P^T  = 2^(S^T scale log2e - LSE2), masked entries 0         (warps 0-7)
+//   dS^T = P^T (dP^T - D_i)                                     (warps 0-7)
 //   dV  += P^T dO       (P^T read from TMEM)                    -> TMEM
 //   dK  += dS^T Q       (dS^T from shared memory)               -> TMEM
 //   dQ^T = K^T dS^T     (per sub-tile)                          -> TMEM -> fp32
-//        vector reductions into a global accumulator            (warps 4-7)
-// Warp 8 issues TMA loads, warp 9 issues the MMAs.  A preprocess kernel forms
-// D_i = dO_i.O_i and the log2-domain LSE and clears the accumulator; a final
-// kernel scales the accumulator into dQ (bf16).
+//        vector reductions into a global accumulator            (warps 8-11)
+// Warps 0-3 / 4-7 each take 32 of the 64 queries of a sub-tile; warp 12 issues
+// the TMA loads, warp 13 the MMAs.  A preprocess kernel forms D_i = dO_i.O_i
+// and the log2-domain LSE (rows padded to whole query tiles) and clears the
+// accumulator; a final kernel scales the accumulator into dQ.  The fp32 path
+// (kind::tf32) transposes its MN-major operands in shared memory (drain warps).
 #include <mutex>
 
 #include "fm_common.cuh"
@@ -137,12 +140,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid (group * T_k, ceil(H / group), B): a group of heads at a time, rank by rank over the
-  // group's heads (rank r takes the key tile with the r-th longest column list); the group is sized
-  // so that its heads' Q, dO and dQ accumulator stay in L2
-  // One CTA per (key tile, K/V head hk).  With grouped-query attention the q_per_kv query heads
-  // hk * q_per_kv + j share this K/V head: their column lists are walked back to back (dK and dV
-  // accumulate over all of them); the list of head j starts at entry hstart[j].
+  // grid (group * T_k, ceil(H_kv / group), B): one CTA per (key tile, K/V head hk); a group of K/V
+  // heads at a time, rank by rank over the group (rank r takes the key tile with the r-th longest
+  // column list), the group sized so that its heads' Q, dO and dQ accumulator stay in L2.  With
+  // grouped-query attention the q_per_kv query heads hk * q_per_kv + j share this K/V head: their
+  // column lists are walked back to back (dK and dV accumulate over all of them); the list of head
+  // j starts at entry hstart[j].
   const int hk = (int)blockIdx.y * p.group + (int)(blockIdx.x % p.group), b = blockIdx.z;
   if (hk >= p.H_kv) return;  // partial last group
   const int G = p.q_per_kv, hq0 = hk * G;

@@ -88,6 +88,14 @@ def workload(config: str, rank: int, masks_arg=None):
     return dict(n=n, B=B, H=H, D=D, masks=specs, desc=desc, seed=1000 * cfg_id + 100000 * rank)
 
 
+def workload_config(wl, world):
+    """The `config` keys both arms report for a workload."""
+    return {"workload": wl["desc"], "B": wl["B"], "H": wl["H"], "seq_len": wl["n"], "head_dim": wl["D"],
+            "masks": [m for m, _ in wl["masks"]],
+            "unmasked_pairs_per_head": [unmasked_pairs(specs, wl["n"]) for _, specs in wl["masks"]],
+            "localize": "8 simulated ranks, dual-chunk, 16 chunks", "parallelism": f"replicas x{world}"}
+
+
 def unmasked_pairs(spec_rows, n):
     """U per batch row from interval lengths (plain per-column count)."""
     out = []
@@ -518,11 +526,9 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), seeded masks)",
-        "config": {"workload": wl["desc"], "B": B, "H": H, "seq_len": n, "head_dim": D,
-                   "masks": [m for m, _ in wl["masks"]], "unmasked_pairs_per_head": U,
-                   "localize": "8 simulated ranks, dual-chunk, 16 chunks", "parallelism": f"replicas x{world}",
-                   "launch": "one CUDA graph per phase, replayed" if graphs_used else "eager",
-                   "l2": "flushed between steps (256 MiB write outside the step events); inputs 256 MiB > L2"},
+        "config": dict(workload_config(wl, world),
+                       launch="one CUDA graph per phase, replayed" if graphs_used else "eager",
+                       l2="flushed between steps (256 MiB write outside the step events); inputs 256 MiB > L2"),
         "fwd": {"effective_tflops": round(fwd_tf, 2), "frac_of_measured_burst": round(fwd_tf / burst, 4),
                 "frac_of_2250_nominal": round(fwd_tf / 2250.0, 4), "ms_per_step": round(fwd_ms / steps, 4)},
         "bwd": {"effective_tflops": round(bwd_tf, 2), "frac_of_measured_burst": round(bwd_tf / burst, 4),
@@ -593,7 +599,7 @@ def run_reference(args):
     return {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), seeded masks)",
-            "config": {"workload": wl["desc"]}, "impl": "reference", "cpu_baseline": cb,
+            "config": workload_config(wl, args.gpus), "impl": "reference", "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

@@ -122,6 +122,27 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
                              fm_mask_meta* out, fm_stream_t stream);
 
 /*
+ * Variable-length batches as one packed sequence (the paper's document masks:
+ * sequences packed end to end attend only within themselves).  Sequence s holds
+ * rows and keys [cu_seqlens[s], cu_seqlens[s+1]); for key j of sequence s:
+ *     LTS[j] = cu_seqlens[s+1], LTE[j] = N   (rows after the sequence are masked)
+ *     UTS[j] = 0, UTE[j] = j if causal, else cu_seqlens[s]   (rows before it)
+ * so the packed call computes, for every sequence, the attention it would get
+ * alone (causal or bidirectional), and every tile between two sequences is a
+ * skip tile.  Keys past cu_seqlens[n_seq] (padding) are masked for all rows.
+ *   cu_seqlens  device int32 [n_seq + 1]: 0 = cu[0] <= cu[1] <= ... <= cu[n_seq] <= N
+ *               (the library reads it on the device and does not check it; an unsorted
+ *               array gives a mask of some other shape, never an out-of-bounds access).
+ *   n_seq       >= 1, <= 2^20;  N >= 1, the packed length (rows = keys = N).
+ *   causal      0 or 1.
+ *   lts..ute    device int32 [N] each (one [B = 1, Hm = 1, N] mask); the attention calls
+ *               want them 16-byte aligned.
+ * Errors: FM_ERR_INVALID_ARG, FM_ERR_CUDA.
+ */
+fm_status fm_varlen_mask(const int32_t* cu_seqlens, int32_t n_seq, int32_t N, int32_t causal, int32_t* lts,
+                         int32_t* lte, int32_t* uts, int32_t* ute, fm_stream_t stream);
+
+/*
  * Clip-shift-max localization (explainer, clip-shift-max / Theorem 1 paragraph:
  * "clip each mark to a chunk, shift it into the rank's concatenated numbering,
  * and take the maximum across the rank's chunks").  For R simulated ranks at
@@ -174,6 +195,9 @@ typedef struct {
   const void* v;
   int32_t H_kv;   /* K/V heads (grouped-query attention): H % H_kv == 0, query head h reads K/V
                      head h / (H / H_kv); 0 means H_kv = H */
+  int32_t deterministic;  /* backward only (the forward always is): 0 = the key tiles add their
+                             dQ contributions in whatever order they finish; 1 = in a fixed order,
+                             so that dQ is bitwise repeatable (see fm_attn_bwd) */
 } fm_attn_args;
 
 /*
@@ -212,6 +236,15 @@ size_t fm_attn_bwd_workspace_bytes(const fm_attn_args* a);
  *   ceil(n_q / 128) <= 4096, else FM_ERR_UNSUPPORTED.
  *   ws       device workspace, ws_bytes >= fm_attn_bwd_workspace_bytes(a), 256-byte
  *            aligned; holds the fp32 dQ accumulator and per-row statistics.
+ *   a->deterministic = 1: the contributions of the key tiles to the fp32 dQ accumulator of a
+ *            query tile are added in ascending key-tile order (each key tile waits, bounded,
+ *            for the ones before it in that tile's row list), so dQ is bitwise the same from
+ *            run to run; dK and dV always are.  Key tiles are then dispatched in ascending
+ *            order rather than longest first, and the workspace grows by
+ *            B * H * ceil(n_k / 128) * ceil(n_q / 128) * 2 + B * H * ceil(n_q / 128) * 4 bytes.
+ *            The order relies on CTAs of lower index starting no later than those of higher
+ *            index; if one waits longer than the bound the call reports FM_ERR_DEVICE_TIMEOUT
+ *            through fm_get_device_status instead of hanging.
  * Errors: FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA.
  */
 fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4],

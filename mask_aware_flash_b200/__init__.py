@@ -49,7 +49,8 @@ class MaskMetaC(ctypes.Structure):
 class AttnArgs(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("n_q", ctypes.c_int32), ("n_k", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("H_kv", ctypes.c_int32)]
+                ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("H_kv", ctypes.c_int32),
+                ("deterministic", ctypes.c_int32)]
 
 
 VecArray = ctypes.c_void_p * 4
@@ -73,6 +74,8 @@ def lib():
         L.fm_localize.restype = ctypes.c_int
         L.fm_kv_chunk_pairs.argtypes = [i32, i32, i32, i32, VecArray, ctypes.POINTER(ctypes.c_int32), i32, vp, vp]
         L.fm_kv_chunk_pairs.restype = ctypes.c_int
+        L.fm_varlen_mask.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp]
+        L.fm_varlen_mask.restype = ctypes.c_int
         L.fm_attn_fwd.argtypes = [ctypes.POINTER(AttnArgs), ctypes.POINTER(MaskMetaC), VecArray, vp, vp, vp]
         L.fm_attn_fwd.restype = ctypes.c_int
         L.fm_attn_bwd_workspace_bytes.argtypes = [ctypes.POINTER(AttnArgs)]
@@ -192,11 +195,23 @@ def fm_kv_chunk_pairs(loc_vecs, n_loc, chunk_len: int, out=None, stream=None):
     return out
 
 
-def _args(q, k, v, scale) -> AttnArgs:
+def fm_varlen_mask(cu_seqlens, N: int, causal: bool = True, out=None, stream=None):
+    """Packed variable-length batch -> the four mask vectors, each int32 [1, 1, N] on the device.
+    cu_seqlens: int32 CUDA tensor [n_seq + 1] of sequence boundaries (0 first, non-decreasing)."""
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise FmError(FM_ERR_INVALID_ARG, "fm_varlen_mask: cu_seqlens must be a contiguous int32 vector")
+    if out is None:
+        out = [torch.empty((1, 1, N), dtype=torch.int32, device=cu_seqlens.device) for _ in range(4)]
+    _check(lib().fm_varlen_mask(_ptr(cu_seqlens), cu_seqlens.numel() - 1, int(N), 1 if causal else 0,
+                                *[_ptr(x) for x in out], _stream(stream)), "fm_varlen_mask")
+    return out
+
+
+def _args(q, k, v, scale, deterministic=False) -> AttnArgs:
     B, n_q, H, D = q.shape
     dtype = 1 if q.dtype == torch.float32 else 0
     return AttnArgs(B, H, n_q, k.shape[1], D, dtype, float(scale), q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                    k.shape[2])
+                    k.shape[2], 1 if deterministic else 0)
 
 
 def fm_attn_fwd(q, k, v, meta: MaskMeta, vecs, scale, o=None, lse=None, stream=None):
@@ -213,15 +228,16 @@ def fm_attn_fwd(q, k, v, meta: MaskMeta, vecs, scale, o=None, lse=None, stream=N
     return o, lse
 
 
-def fm_attn_bwd_workspace_bytes(q, k, v, scale=1.0) -> int:
-    a = _args(q, k, v, scale)
+def fm_attn_bwd_workspace_bytes(q, k, v, scale=1.0, deterministic=False) -> int:
+    a = _args(q, k, v, scale, deterministic)
     return int(lib().fm_attn_bwd_workspace_bytes(ctypes.byref(a)))
 
 
 def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=None, dv=None, ws=None,
-                stream=None):
-    """Gradients (dtype of q) of the masked attention; ws: optional uint8 CUDA workspace."""
-    a = _args(q, k, v, scale)
+                stream=None, deterministic=False):
+    """Gradients (dtype of q) of the masked attention; ws: optional uint8 CUDA workspace.
+    deterministic: add the key tiles' dQ contributions in a fixed order (bitwise repeatable dQ)."""
+    a = _args(q, k, v, scale, deterministic)
     nbytes = lib().fm_attn_bwd_workspace_bytes(ctypes.byref(a))
     if ws is None:
         ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device)

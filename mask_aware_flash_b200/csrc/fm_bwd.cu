@@ -41,7 +41,10 @@ constexpr float kPosInf = __builtin_huge_valf();
 struct BwdParams {
   const int32_t* col_count;    // [B, Hm, T_k]
   const int32_t* col_entries;  // [B, Hm, T_k, T_q]
-  const int32_t* order;        // [B, Hm, T_k] dispatch order (longest first)
+  const int32_t* order;        // [B, Hm, T_k] dispatch order (longest first); null = ascending
+  const uint16_t* turn;        // fixed-order dQ: [B, Hm, T_k, T_q] position of key tile kt in the
+                               // row list of query tile qt; null = unordered adds
+  int* dq_sem;                 // fixed-order dQ: [B, H, T_q] key tiles added so far per query tile
   const int32_t* vec[4];       // [B, Hm, n_k] or null
   const float* lse2;           // [B, H, n_q] log2-domain LSE, +inf on empty rows
   const float* dvec;           // [B, H, n_q] D_i = dO_i . O_i
@@ -74,7 +77,8 @@ struct BwdSmem {
   static constexpr int kDS = kDO + kQStages * kQStage;  // kDSBufs buffers
   static constexpr int kStats = kDS + kDSBufs * kDSBytes;  // kQStages x (64 lse2 + 64 D_i) fp32
   static constexpr int kList = kStats + kQStages * 2 * kBQ * 4;  // column list, uint16
-  static constexpr int kHeads = kList + kMaxList * 2;  // [q_per_kv + 1] list offsets, int32 (<= 65)
+  static constexpr int kTurn = kList + kMaxList * 2;  // fixed-order dQ: turn of each list entry, uint16
+  static constexpr int kHeads = kTurn + kMaxList * 2;  // [q_per_kv + 1] list offsets, int32 (<= 65)
   static constexpr int kBar = kHeads + 65 * 4 + 12;      // (8-byte aligned)
   enum { KV_FULL, QDO_FULL0, QDO_FULL1, QDO_FULL2, QDO_EMPTY0, QDO_EMPTY1, QDO_EMPTY2, SDP_FULL, DP_FREE,
          DS_READY, DS_EMPTY0, DS_EMPTY1, DQ_FULL, DQ_EMPTY, ACC_FULL, DRAIN,
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (hk >= p.H_kv) return;  // partial last group
   const int G = p.q_per_kv, hq0 = hk * G;
   auto bhm_of = [&](int hq) -> int64_t { return (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : hq); };
-  const int kt = __ldg(p.order + bhm_of(hq0) * p.T_k + blockIdx.x / p.group);
+  const int kt = p.order ? __ldg(p.order + bhm_of(hq0) * p.T_k + blockIdx.x / p.group) : (int)(blockIdx.x / p.group);
   int cnt = 0;  // entries over the group's query heads
   for (int jq = 0; jq < G; ++jq) cnt += __ldg(p.col_count + bhm_of(hq0 + jq) * p.T_k + kt);
   const int nsub = 2 * cnt;  // two 64-row sub-tiles per listed 128-row query tile
@@ -176,7 +180,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     *abort_flag = 0;
     misc[2] = 0;
     fence_barrier_init();
-    if (cnt > 0) {  // K and V first: their latency overlaps the list copy and the TMEM allocation
+    {  // K and V first (as soon as the key tile is known): their latency overlaps the list copy and
+       // the TMEM allocation.  A CTA with an empty list waits for them before it exits.
       fence_proxy_async_smem();
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -188,14 +193,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   }
   int* hstart = reinterpret_cast<int*>(smem + S::kHeads);  // [G + 1]
+  uint16_t* turn = reinterpret_cast<uint16_t*>(smem + S::kTurn);
   {
+    // Fixed-order dQ walks each list from the last query tile down, so that the key tiles of a
+    // head, which all start their lists at about the same time, reach a shared query tile in
+    // ascending order a few adds apart rather than a whole list apart.
+    const bool rev = p.turn != nullptr;
     int start = 0;
     for (int jq = 0; jq < G; ++jq) {
       const int64_t bj = bhm_of(hq0 + jq);
       const int cj = __ldg(p.col_count + bj * p.T_k + kt);
       const int32_t* ej = p.col_entries + (bj * p.T_k + kt) * p.T_q;
       if (threadIdx.x == 0) hstart[jq] = start;
-      for (int t = threadIdx.x; t < cj; t += kBwdThreads) list[start + t] = (uint16_t)__ldg(ej + t);
+      for (int t = threadIdx.x; t < cj; t += kBwdThreads) {
+        const int32_t e = __ldg(ej + (rev ? cj - 1 - t : t));
+        list[start + t] = (uint16_t)e;
+        if (rev) turn[start + t] = __ldg(p.turn + (bj * p.T_k + kt) * p.T_q + (e >> 1));
+      }
       start += cj;
     }
     if (threadIdx.x == 0) hstart[G] = start;
@@ -237,7 +251,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         const int q0 = sub_q0(i);
-        const int hq = hq0 + head_of(i, jh);
+        const int hq = hq0 + (G > 1 ? head_of(i, jh) : 0);
         const int64_t bh = (int64_t)b * p.H + hq;
         const uint32_t fb = bar(S::QDO_FULL0 + st);
         mbar_arrive_expect_tx(fb, 2 * S::kQStage + 2 * kBQ * 4);
@@ -386,18 +400,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int64_t j = (int64_t)kt * kTile + r;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const bool no_key = j >= p.n_k;  // past a ragged n_k: a zero-filled key row, masked for every query
-    int32_t lts = p.n_q, lte = p.n_q, uts = 0, ute = 0;
-    int jh = 0, jv = -1;  // head cursor; head whose vectors are loaded
+    int32_t lts, lte, uts, ute;
+    auto load_bounds = [&](int jq) {  // this key's bounds for query head hq0 + jq
+      const int64_t voff = bhm_of(hq0 + jq) * p.n_k + j;
+      lts = (p.vec[0] && !no_key) ? __ldg(p.vec[0] + voff) : p.n_q;
+      lte = (p.vec[1] && !no_key) ? __ldg(p.vec[1] + voff) : p.n_q;
+      uts = (p.vec[2] && !no_key) ? __ldg(p.vec[2] + voff) : 0;
+      ute = (p.vec[3] && !no_key) ? __ldg(p.vec[3] + voff) : 0;
+    };
+    load_bounds(0);
+    const bool per_head = G > 1 && p.Hm != 1;  // grouped query heads with masks of their own
+    int jh = 0, jv = 0;  // head cursor; head whose bounds are loaded
     bool ok = true;
     for (int i = 0; i < nsub; ++i) {
-      const int jq = head_of(i, jh);
-      if (jv < 0 || (p.Hm != 1 && jq != jv)) {  // this key's bounds for the sub-tile's query head
-        const int64_t voff = bhm_of(hq0 + jq) * p.n_k + j;
-        lts = (p.vec[0] && !no_key) ? __ldg(p.vec[0] + voff) : p.n_q;
-        lte = (p.vec[1] && !no_key) ? __ldg(p.vec[1] + voff) : p.n_q;
-        uts = (p.vec[2] && !no_key) ? __ldg(p.vec[2] + voff) : 0;
-        ute = (p.vec[3] && !no_key) ? __ldg(p.vec[3] + voff) : 0;
-        jv = jq;
+      if (per_head) {
+        const int jq = head_of(i, jh);
+        if (jq != jv) {
+          load_bounds(jq);
+          jv = jq;
+        }
       }
       const int st = i % NS, bi = i % NDS, sb = i & 1;  // Q/dO stage, dS^T buffer, S^T buffer
       const int q0 = sub_q0(i) + c0;
@@ -498,7 +519,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int i = 0; ok && i < nsub; ++i) {
       const int q0 = sub_q0(i);
-      float* acc_bh = p.dq_acc + ((int64_t)b * p.H + hq0 + head_of(i, jh)) * (int64_t)p.n_q_pad * D;
+      const int64_t bh = (int64_t)b * p.H + hq0 + (G > 1 ? head_of(i, jh) : 0);
+      float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q_pad * D;
       if constexpr (F32) {
         const int st = i % NS;
         ok = all_drain_threads(mbar_wait(bar(S::QT_GO0 + st), (i / NS) & 1, abort_flag));
@@ -515,12 +537,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_ld64(tdQ + lane_addr, a);
       tc_fence_before();
       mbar_arrive(bar(S::DQ_EMPTY));
+      int* sem = p.dq_sem ? p.dq_sem + bh * p.T_q + (q0 >> 7) : nullptr;
+      if (sem && (i & 1) == 0) {  // fixed order: wait until the key tiles before this one have added
+        ok = all_drain_threads(d != 0 || flag_wait_eq(sem, turn[i >> 1], p.status, abort_flag));
+        if (!ok) break;
+      }
       if (d < D) {
         float* blk = acc_bh + (int64_t)q0 * D;  // [16 groups of 4 queries][D][4]
 #pragma unroll
         for (int g = 0; g < 16; ++g)
           red_add_v4(blk + (g * D + d) * 4, __uint_as_float(a[4 * g]), __uint_as_float(a[4 * g + 1]),
                      __uint_as_float(a[4 * g + 2]), __uint_as_float(a[4 * g + 3]));
+      }
+      if (sem && (i & 1) == 1) {  // both sub-tiles added: pass the query tile on to the next key tile
+        all_drain_threads(true);
+        if (d == 0) st_release_gpu(sem, turn[i >> 1] + 1);
       }
     }
     if (!ok) record_failure(p.status, abort_flag, 14);
@@ -581,6 +612,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   }
 
+  if (threadIdx.x == 0 && cnt == 0) mbar_wait(bar(S::KV_FULL), 0, never);  // no copy in flight at exit
   tc_fence_before();
   __syncthreads();
   if (warp == 13) {
@@ -595,7 +627,7 @@ template <int D, bool F32>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ o, const void* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ dvec, float* __restrict__ acc, int B,
-                                                       int H, int n_q, int n_q_pad) {
+                                                       int H, int n_q, int n_q_pad, int* __restrict__ dq_sem) {
   const int64_t rows = (int64_t)B * n_q * H;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t < rows) {
@@ -645,6 +677,25 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ 
   float4* a4 = reinterpret_cast<float4*>(acc);
   const int64_t n4 = (int64_t)B * H * n_q_pad * D / 4;
   for (int64_t k = t; k < n4; k += stride) a4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (dq_sem)  // fixed-order dQ: no key tile has added yet
+    for (int64_t k = t; k < (int64_t)B * H * (n_q_pad / kTile); k += stride) dq_sem[k] = 0;
+}
+
+// Fixed-order dQ: turn[bhm, kt, qt] = position of key tile kt in the row list of query tile qt
+// (the number of non-skip key tiles before it), one warp per row list.  Entries of skip pairs
+// are never read and stay unwritten.
+__global__ void __launch_bounds__(256) bwd_turn_kernel(const int32_t* __restrict__ row_count,
+                                                       const int32_t* __restrict__ row_entries,
+                                                       uint16_t* __restrict__ turn, int BHm, int T_q, int T_k) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (int64_t)BHm * T_q) return;
+  const int64_t bhm = w / T_q;
+  const int qt = (int)(w % T_q);
+  const int c = __ldg(row_count + w);
+  const int32_t* e = row_entries + w * T_k;
+  for (int pos = lane; pos < c; pos += 32)
+    turn[(bhm * T_k + (__ldg(e + pos) >> 1)) * T_q + qt] = (uint16_t)pos;
 }
 
 // dQ[b, i, h, :] = scale * acc for one 64-row block per CTA: the block (a
@@ -688,16 +739,24 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct BwdLayout {
-  size_t acc, lse2, dvec, total;
+  size_t acc, lse2, dvec, turn, sem, total;
 };
 
+// Workspace: fp32 dQ accumulator, log2 LSE and D_i per padded row; for fixed-order dQ also the
+// turn table (sized for Hm = H, the larger of the two mask-head counts) and one counter per
+// query tile.
 BwdLayout bwd_layout(const fm_attn_args* a) {
   BwdLayout L;
-  const size_t rows = (size_t)a->B * a->H * (((size_t)a->n_q + kTile - 1) / kTile * kTile);  // padded rows
+  const size_t T_q = ((size_t)a->n_q + kTile - 1) / kTile, T_k = ((size_t)a->n_k + kTile - 1) / kTile;
+  const size_t rows = (size_t)a->B * a->H * T_q * kTile;  // padded rows
   L.acc = 0;
   L.lse2 = align256(rows * a->D * 4);
   L.dvec = L.lse2 + align256(rows * 4);
-  L.total = L.dvec + align256(rows * 4);
+  L.turn = L.sem = L.total = L.dvec + align256(rows * 4);
+  if (a->deterministic) {
+    L.sem = L.turn + align256((size_t)a->B * a->H * T_k * T_q * 2);
+    L.total = L.sem + align256((size_t)a->B * a->H * T_q * 4);
+  }
   return L;
 }
 
@@ -711,6 +770,8 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   float* acc = reinterpret_cast<float*>(w + L.acc);
   float* lse2 = reinterpret_cast<float*>(w + L.lse2);
   float* dvec = reinterpret_cast<float*>(w + L.dvec);
+  uint16_t* turn = a->deterministic ? reinterpret_cast<uint16_t*>(w + L.turn) : nullptr;
+  int* dq_sem = a->deterministic ? reinterpret_cast<int*>(w + L.sem) : nullptr;
   const int H_kv = a->H_kv ? a->H_kv : a->H;
   CUtensorMap tq, tdo, tk, tv, tdk, tdv;
   auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
@@ -720,11 +781,13 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
     return FM_ERR_CUDA;
   const int64_t rows = (int64_t)a->B * a->n_q * a->H;
   bwd_prep_kernel<D, F32><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(o, dout, lse, lse2, dvec, acc, a->B,
-      a->H, a->n_q, (a->n_q + kTile - 1) / kTile * kTile);
+      a->H, a->n_q, (a->n_q + kTile - 1) / kTile * kTile, dq_sem);
   BwdParams p;
   p.col_count = meta->col_count;
   p.col_entries = meta->col_entries;
-  p.order = meta->bwd_order;
+  p.order = turn ? nullptr : meta->bwd_order;  // fixed order: key tiles in ascending order
+  p.turn = turn;
+  p.dq_sem = dq_sem;
   for (int c = 0; c < 4; ++c) p.vec[c] = vec ? vec[c] : nullptr;
   p.lse2 = lse2;
   p.dvec = dvec;
@@ -747,6 +810,11 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   p.scale = a->scale;
   p.scale_log2 = a->scale * 1.4426950408889634f;
   if (!smem_opt_in<bwd_kernel<D, F32>>(S::kAlloc)) return FM_ERR_CUDA;
+  if (turn) {
+    const int64_t warps = (int64_t)a->B * meta->d.Hm * p.T_q;
+    bwd_turn_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(meta->row_count, meta->row_entries, turn,
+                                                                    a->B * meta->d.Hm, p.T_q, p.T_k);
+  }
   bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H_kv + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
   bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (p.n_q_pad / 64)), 256, 0, stream>>>(
       acc, dq, a->B, a->H, a->n_q, p.n_q_pad, a->scale);

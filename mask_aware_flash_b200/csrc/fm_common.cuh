@@ -491,6 +491,32 @@ __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
+// Ordered hand-off between CTAs through a global counter (acquire / release at GPU scope).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait until *flag == want.  Gives up (false) after kTimeoutNs, when the CTA's abort flag
+// is raised, or when the device status word shows that some kernel has already failed (so that
+// the CTAs queued behind a failed one do not each wait out the bound).
+__device__ __forceinline__ bool flag_wait_eq(const int* flag, int want, const int* status,
+                                             const volatile int* abort) {
+  if (ld_acquire_gpu(flag) == want) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) == want) return true;
+    if ((it & 15u) == 0) {
+      if (*abort || (status && *reinterpret_cast<const volatile int*>(status) != 0)) return false;
+      if (globaltimer() - t0 > kTimeoutNs) return false;
+    }
+  }
+}
+
 __device__ __forceinline__ int ld_nc_i32(const int32_t* p) {
   int v;
   asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));

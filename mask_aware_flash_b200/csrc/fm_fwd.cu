@@ -634,6 +634,7 @@ fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const
   if (d.Hm != 1 && d.Hm != a->H) return FM_ERR_INVALID_ARG;
   const int H_kv = a->H_kv ? a->H_kv : a->H;  // grouped-query attention: H_kv divides H
   if (H_kv < 1 || H_kv > a->H || a->H % H_kv) return FM_ERR_INVALID_ARG;
+  if (a->deterministic != 0 && a->deterministic != 1) return FM_ERR_INVALID_ARG;
   if (a->H / H_kv > 64) return FM_ERR_UNSUPPORTED;  // the backward's per-CTA head table
   if (!meta->row_count || !meta->row_entries || !meta->col_count || !meta->col_entries || !meta->fwd_order ||
       !meta->bwd_order)

@@ -132,6 +132,32 @@ __global__ void __launch_bounds__(256) meta_lists_kernel(const MetaParams p) {
   }
 }
 
+// Packed variable-length batch -> document-mask vectors, one thread per key: the key's sequence is
+// the largest s < n_seq with cu[s] <= j (binary search; empty sequences are passed over).
+__global__ void __launch_bounds__(256) varlen_mask_kernel(const int32_t* __restrict__ cu, int n_seq, int N,
+                                                          int causal, int32_t* __restrict__ lts,
+                                                          int32_t* __restrict__ lte, int32_t* __restrict__ uts,
+                                                          int32_t* __restrict__ ute) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= N) return;
+  const int j = (int)t;
+  int l0 = 0, l1 = N, u1 = 0;  // a padding key past the last sequence: every row masked
+  if (j < __ldg(cu + n_seq)) {
+    int lo = 0, hi = n_seq - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(cu + mid) <= j) lo = mid;
+      else hi = mid - 1;
+    }
+    l0 = __ldg(cu + lo + 1);             // rows after the sequence
+    u1 = causal ? j : __ldg(cu + lo);    // rows before the key (causal) or before the sequence
+  }
+  lts[j] = l0;
+  lte[j] = l1;
+  uts[j] = 0;
+  ute[j] = u1;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Dispatch orders for the attention kernels (longest first).  One CTA per
@@ -265,6 +291,20 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
   const int64_t warps_l = (int64_t)p.BHm * (p.T_q > p.T_k ? p.T_q : p.T_k);
   fm::meta_lists_kernel<<<dim3((unsigned)((warps_l + 7) / 8), 2), 256, 0, s>>>(p);
   fm::meta_order_kernel<<<dim3((unsigned)p.BHm, 2), 1024, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
+}
+
+fm_status fm_varlen_mask(const int32_t* cu_seqlens, int32_t n_seq, int32_t N, int32_t causal, int32_t* lts,
+                         int32_t* lte, int32_t* uts, int32_t* ute, fm_stream_t stream) {
+  if (!cu_seqlens || !lts || !lte || !uts || !ute || n_seq < 1 || n_seq > (1 << 20) || N < 1 ||
+      (causal != 0 && causal != 1))
+    return FM_ERR_INVALID_ARG;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(cu_seqlens) | reinterpret_cast<uintptr_t>(lts) |
+                       reinterpret_cast<uintptr_t>(lte) | reinterpret_cast<uintptr_t>(uts) |
+                       reinterpret_cast<uintptr_t>(ute);
+  if (al & 3) return FM_ERR_INVALID_ARG;
+  fm::varlen_mask_kernel<<<(unsigned)(((int64_t)N + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      cu_seqlens, n_seq, N, causal, lts, lte, uts, ute);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

@@ -99,6 +99,25 @@ def kv_chunk_pairs(n_q, n_k, chunk_len, lts, lte, uts, ute) -> np.ndarray:
     return out
 
 
+def varlen_vectors(cu_seqlens, N, causal) -> list:
+    """[explainer] document masks: sequences packed end to end, each attending
+    only within itself (causal or bidirectional).  Sequence s owns positions
+    [cu[s], cu[s+1]).  Its keys mask the rows after the sequence through the lower
+    stretch [cu[s+1], N) and, through the upper stretch [0, UTE), the rows before
+    the key (causal: UTE = j) or before the sequence (UTE = cu[s]).  Reading:
+    keys past cu[-1] (padding) mask every row ([0, N) as the lower stretch)."""
+    cu = [int(x) for x in cu_seqlens]
+    lts = np.zeros(N, np.int32)
+    lte = np.full(N, N, np.int32)
+    uts = np.zeros(N, np.int32)
+    ute = np.zeros(N, np.int32)
+    for s in range(len(cu) - 1):
+        for j in range(cu[s], cu[s + 1]):
+            lts[j] = cu[s + 1]
+            ute[j] = j if causal else cu[s]
+    return [lts, lte, uts, ute]
+
+
 def tile_meta(n_q, n_k, lts, lte, uts, ute, tile_q=128, tile_k=128) -> dict:
     """[explainer] tile paragraph: per-key-tile min/max of the four vectors,
     class of every (query tile, key tile) pair (0 skip, 1 partial, 2 full) and

@@ -141,6 +141,26 @@ def test_bwd_rejects_before_launch(L):
         fm.FM_ERR_UNSUPPORTED
 
 
+def test_deterministic_flag(L):
+    """Fixed-order dQ: the flag is 0 or 1, and its workspace adds the turn table (2 bytes per
+    (b, h, key tile, query tile)) and one int32 counter per (b, h, query tile), each 256-aligned."""
+    vec = fm.VecArray(None, None, None, None)
+    p = [ctypes.c_void_p(0x100000 * (t + 1)) for t in range(6)]
+    a, m = _attn(L, n_q=384, n_k=640, H=2)
+    base = L.fm_attn_bwd_workspace_bytes(ctypes.byref(a))
+    a.deterministic = 1
+    det = L.fm_attn_bwd_workspace_bytes(ctypes.byref(a))
+    al = lambda x: (x + 255) // 256 * 256
+    assert det - base == al(1 * 2 * 5 * 3 * 2) + al(1 * 2 * 3 * 4)
+    assert L.fm_attn_bwd(ctypes.byref(a), ctypes.byref(m), vec, *p, ctypes.c_void_p(0x900000), base, None) == \
+        fm.FM_ERR_WORKSPACE  # the deterministic call needs the larger workspace
+    a.deterministic = 2
+    assert L.fm_attn_bwd(ctypes.byref(a), ctypes.byref(m), vec, *p, ctypes.c_void_p(0x900000), det, None) == \
+        fm.FM_ERR_INVALID_ARG
+    assert L.fm_attn_fwd(ctypes.byref(a), ctypes.byref(m), vec, ctypes.c_void_p(0x50000),
+                         ctypes.c_void_p(0x60000), None) == fm.FM_ERR_INVALID_ARG
+
+
 def test_no_oracle_import_in_library():
     """The product path must not reach the oracle or any CPU fallback."""
     pkg = os.path.join(ROOT, "mask_aware_flash_b200")
@@ -169,3 +189,13 @@ def test_kv_chunk_pairs_rejects_bad_args(L):
     many = np.full(256, 64, np.int32)
     assert L.fm_kv_chunk_pairs(300, 1, 256, 256, vec, many.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), 64, out,
                                None) == fm.FM_ERR_UNSUPPORTED  # 256 ranks x 300 rows > 65535
+
+
+def test_varlen_mask_rejects_bad_args(L):
+    cu, o = ctypes.c_void_p(0x10000), [ctypes.c_void_p(0x20000 * (t + 1)) for t in range(4)]
+    assert L.fm_varlen_mask(None, 2, 100, 1, *o, None) == fm.FM_ERR_INVALID_ARG
+    assert L.fm_varlen_mask(cu, 0, 100, 1, *o, None) == fm.FM_ERR_INVALID_ARG        # no sequence
+    assert L.fm_varlen_mask(cu, 2, 0, 1, *o, None) == fm.FM_ERR_INVALID_ARG          # empty pack
+    assert L.fm_varlen_mask(cu, 2, 100, 2, *o, None) == fm.FM_ERR_INVALID_ARG        # causal flag
+    assert L.fm_varlen_mask(cu, 2, 100, 1, o[0], o[1], ctypes.c_void_p(0x60002), o[3], None) == \
+        fm.FM_ERR_INVALID_ARG  # misaligned int32 output

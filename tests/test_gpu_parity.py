@@ -195,7 +195,7 @@ def test_chunk_costs_and_balanced_assignment(fm):
 
 
 # ---------------------------------------------------------------------------- attention
-def _run_attention(fm, B, H, n_q, n_k, D, vecs_np, Hm, seed, scale=None, bwd=True):
+def _run_attention(fm, B, H, n_q, n_k, D, vecs_np, Hm, seed, scale=None, bwd=True, det=False):
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     host, dev = _inputs(B, n_q, n_k, H, D, seed)
     vt = [None if v is None else torch.from_numpy(np.ascontiguousarray(v, np.int32)).cuda() for v in vecs_np]
@@ -203,8 +203,8 @@ def _run_attention(fm, B, H, n_q, n_k, D, vecs_np, Hm, seed, scale=None, bwd=Tru
     o, lse = fm.fm_attn_fwd(dev[0], dev[1], dev[2], meta, vt, scale)
     res = {"o": o, "lse": lse, "host": host, "meta": meta, "vt": vt, "scale": scale}
     if bwd:
-        dq, dk, dv = fm.fm_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], meta, vt, scale)
-        res.update(dq=dq, dk=dk, dv=dv)
+        dq, dk, dv = fm.fm_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], meta, vt, scale, deterministic=det)
+        res.update(dq=dq, dk=dk, dv=dv, dev=dev)
     torch.cuda.synchronize()
     assert fm.fm_get_device_status() == 0
     return res
@@ -326,8 +326,9 @@ def test_ragged_fp32(fm):
     _compare(_run_fp32(fm, 1, 2, n, vecs, 66), vecs, 1)
 
 
-@pytest.mark.parametrize("H,H_kv,Hm,D", [(4, 2, 1, 128), (4, 1, 1, 64), (6, 2, 6, 128), (8, 8, 1, 64)])
-def test_grouped_query_heads(fm, H, H_kv, Hm, D):
+@pytest.mark.parametrize("H,H_kv,Hm,D,det", [(4, 2, 1, 128, False), (4, 1, 1, 64, False), (6, 2, 6, 128, False),
+                                             (8, 8, 1, 64, False), (6, 2, 6, 128, True)])
+def test_grouped_query_heads(fm, H, H_kv, Hm, D, det):
     """Grouped-query attention: K / V have H_kv heads, query head h reads K/V head h // (H / H_kv).
     The oracle sees K / V repeated to H heads; the reference dK / dV of a K/V head is the sum over
     its query heads of their gradients (the plain chain rule through the repetition)."""
@@ -345,7 +346,7 @@ def test_grouped_query_heads(fm, H, H_kv, Hm, D):
     scale = 1.0 / math.sqrt(D)
     meta = fm.fm_build_mask_meta(*vt, n_q=n)
     o, lse = fm.fm_attn_fwd(dev[0], dev[1], dev[2], meta, vt, scale)
-    dq, dk, dv = fm.fm_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], meta, vt, scale)
+    dq, dk, dv = fm.fm_attn_bwd(dev[0], dev[1], dev[2], o, lse, dev[3], meta, vt, scale, deterministic=det)
     torch.cuda.synchronize()
     assert fm.fm_get_device_status() == 0
     assert dk.shape == (1, n, H_kv, D)
@@ -368,6 +369,42 @@ def test_grouped_query_heads(fm, H, H_kv, Hm, D):
             e = exp[:, hk]
             err = np.abs(got.float().cpu().numpy()[0, :, hk] - e).max() / max(np.abs(e).max(), 1e-30)
             assert err <= G_TOL, f"{name} head {hk}: rel-to-max {err}"
+
+
+@pytest.mark.parametrize("family,n,B,H,D", [("causal_document", 1000, 2, 3, 128), ("global_sliding", 2048, 1, 2, 64),
+                                             ("random_eviction", 1536, 1, 4, 128)])
+def test_fixed_order_dq(fm, family, n, B, H, D):
+    """deterministic=1: dQ matches the oracle, and three backward calls on the same inputs give
+    bitwise identical dQ, dK and dV (each query tile takes its key tiles' contributions in
+    ascending key-tile order)."""
+    vecs = _vec_stack(synth.make_family(family, n, 93), B, 1)
+    res = _run_attention(fm, B, H, n, n, D, vecs, 1, seed=94, det=True)
+    _compare(res, vecs, 1)
+    q, k, v, do = res["dev"]
+    for _ in range(2):
+        again = fm.fm_attn_bwd(q, k, v, res["o"], res["lse"], do, res["meta"], res["vt"], res["scale"],
+                               deterministic=True)
+        torch.cuda.synchronize()
+        assert fm.fm_get_device_status() == 0
+        for name, a, b in zip(("dq", "dk", "dv"), (res["dq"], res["dk"], res["dv"]), again):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"{name} differs between calls"
+
+
+def test_fully_masked_key_tile(fm):
+    """Keys 128..255 masked for every row: that key tile has an empty column list (no MMA work),
+    its dK / dV are exactly 0, and the other tiles still match the oracle."""
+    n_q, n_k = 256, 512
+    lts = np.full(n_k, n_q, np.int32)
+    lte = np.full(n_k, n_q, np.int32)
+    lts[128:256], lte[128:256] = 0, n_q
+    uts = np.zeros(n_k, np.int32)
+    ute = np.minimum(np.arange(n_k), n_q).astype(np.int32)  # causal on the remaining keys
+    vecs = [x[None, None] for x in (lts, lte, uts, ute)]
+    res = _run_attention(fm, 1, 2, n_q, n_k, 128, vecs, 1, seed=91)
+    assert int(res["meta"].col_count[0, 0, 1].item()) == 0
+    _compare(res, vecs, 1)
+    assert np.all(res["dk"].float().cpu().numpy()[0, 128:256] == 0.0)
+    assert np.all(res["dv"].float().cpu().numpy()[0, 128:256] == 0.0)
 
 
 def test_dead_rows_and_cross_lengths(fm):
@@ -454,3 +491,42 @@ def test_localized_forward_equals_global_rows(fm):
         assert torch.equal(lo, go[:, rows]), f"rank {r}: O differs"
         assert torch.equal(llse, glse[:, :, rows]), f"rank {r}: LSE differs"
     assert fm.fm_get_device_status() == 0
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_packed_batch(fm, causal):
+    """A packed variable-length batch (one empty sequence, a padding tail past the last one):
+    fm_varlen_mask matches the oracle's vectors bit for bit, the packed attention matches the
+    oracle, and each sequence's rows match the same sequence run on its own (causal or unmasked),
+    so the packing is invisible to the result."""
+    N, H, D = 1500, 2, 128
+    cu = np.array([0, 200, 712, 712, 1000, 1392], np.int32)  # sequence 2 is empty; keys 1392.. pad
+    vecs_dev = fm.fm_varlen_mask(torch.from_numpy(cu).cuda(), N, causal=causal)
+    torch.cuda.synchronize()
+    ref_vecs = oracle.varlen_vectors(cu, N, causal)
+    for got, exp in zip(vecs_dev, ref_vecs):
+        np.testing.assert_array_equal(got.cpu().numpy()[0, 0], exp)
+    vecs = [x[None, None] for x in ref_vecs]
+    res = _run_attention(fm, 1, H, N, N, D, vecs, 1, seed=95)
+    _compare(res, vecs, 1)
+    assert np.all(np.isneginf(res["lse"].cpu().numpy()[0, :, 1392:]))  # padding rows see no key
+    q, k, v, do = res["dev"]
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        if a == b:
+            continue
+        L = b - a
+        alone = [np.full(L, L), np.full(L, L), np.zeros(L), np.arange(L) if causal else np.zeros(L)]
+        vt = [torch.from_numpy(x.astype(np.int32)[None, None]).cuda() for x in alone]
+        meta = fm.fm_build_mask_meta(*vt, n_q=L)
+        qs, ks, vs, dos = (x[:, a:b].contiguous() for x in (q, k, v, do))
+        o, lse = fm.fm_attn_fwd(qs, ks, vs, meta, vt, res["scale"])
+        dq, dk, dv = fm.fm_attn_bwd(qs, ks, vs, o, lse, dos, meta, vt, res["scale"])
+        torch.cuda.synchronize()
+        assert fm.fm_get_device_status() == 0
+        assert (o.float() - res["o"][:, a:b].float()).abs().max().item() <= O_TOL
+        assert (lse - res["lse"][:, :, a:b]).abs().max().item() <= LSE_TOL
+        for name, alone, packed in (("dq", dq, res["dq"]), ("dk", dk, res["dk"]), ("dv", dv, res["dv"])):
+            p = packed[:, a:b].float()
+            err = (alone.float() - p).abs().max().item() / max(p.abs().max().item(), 1e-30)
+            assert err <= G_TOL, f"{name} of sequence {s}: {err}"

@@ -315,3 +315,37 @@ def test_kv_chunk_pairs_ranks_partition_global():
         np.testing.assert_array_equal(total, glob)
         assert glob.sum() == oracle.count_unmasked_dense(N, N, *vecs)
     assert pruned > 0  # the cases include chunks some ranks never need
+
+
+def _varlen_predicate(cu, N, causal):
+    """Plain definition of a packed batch: (i, j) is visible iff both lie in the same sequence
+    and, when causal, j <= i; every other pair (other sequence, padding) is masked."""
+    seq = np.full(N, -1)
+    for s in range(len(cu) - 1):
+        seq[cu[s]:cu[s + 1]] = s
+    i, j = np.arange(N)[:, None], np.arange(N)[None, :]
+    visible = (seq[:, None] == seq[None, :]) & (seq[:, None] >= 0)
+    if causal:
+        visible &= j <= i
+    return ~visible
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_vectors_match_packed_predicate(causal):
+    r = np.random.default_rng(41)
+    for N in (1, 7, 130, 300, 517):
+        for _ in range(20):
+            n_seq = int(r.integers(1, 9))
+            cuts = np.sort(r.integers(0, N + 1, n_seq))  # repeated cuts = empty sequences
+            cu = np.concatenate([[0], cuts])
+            vecs = oracle.varlen_vectors(cu, N, causal)
+            np.testing.assert_array_equal(oracle.dense_mask(N, N, *vecs), _varlen_predicate(cu, N, causal))
+
+
+def test_varlen_single_sequence_is_causal_or_full():
+    """One sequence over all N positions: the causal mask (UTE = j) or no mask at all."""
+    N = 300
+    lts, lte, uts, ute = oracle.varlen_vectors([0, N], N, True)
+    assert oracle.count_unmasked(N, N, lts, lte, uts, ute) == N * (N + 1) // 2
+    np.testing.assert_array_equal(ute, np.arange(N))
+    assert oracle.count_unmasked(N, N, *oracle.varlen_vectors([0, N], N, False)) == N * N

@@ -199,3 +199,11 @@ def test_varlen_mask_rejects_bad_args(L):
     assert L.fm_varlen_mask(cu, 2, 100, 2, *o, None) == fm.FM_ERR_INVALID_ARG        # causal flag
     assert L.fm_varlen_mask(cu, 2, 100, 1, o[0], o[1], ctypes.c_void_p(0x60002), o[3], None) == \
         fm.FM_ERR_INVALID_ARG  # misaligned int32 output
+
+
+def test_varlen_binding_rejects_non_int32():
+    torch = pytest.importorskip("torch")
+    with pytest.raises(fm.FmError):
+        fm.fm_varlen_mask(torch.zeros(3, dtype=torch.int64), 10)
+    with pytest.raises(fm.FmError):
+        fm.fm_varlen_mask(torch.zeros((2, 2), dtype=torch.int32), 10)

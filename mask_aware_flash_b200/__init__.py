@@ -10,8 +10,9 @@ Entry points (same names as the C ABI):
   fm_build_mask_meta(lts, lte, uts, ute, n_q)      -> MaskMeta
   fm_localize(vecs, chunk_start, chunk_len)         -> 4 tensors [R, B, Hm, N]
   fm_kv_chunk_pairs(loc_vecs, n_loc, chunk_len)     -> int64 [R, B, Hm, n_chunks]
+  fm_varlen_mask(cu_seqlens, N, causal)             -> 4 tensors [1, 1, N]
   fm_attn_fwd(q, k, v, meta, vecs, scale)           -> (o, lse)
-  fm_attn_bwd(q, k, v, o, lse, do, meta, vecs, scale) -> (dq, dk, dv)
+  fm_attn_bwd(q, k, v, o, lse, do, meta, vecs, scale, deterministic=False) -> (dq, dk, dv)
 """
 from __future__ import annotations
 
@@ -245,7 +246,8 @@ def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=No
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     _check(lib().fm_attn_bwd(ctypes.byref(a), ctypes.byref(meta.c), _vecs(vecs), _ptr(o), _ptr(lse), _ptr(do),
-                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)), "fm_attn_bwd")
+                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "fm_attn_bwd")
     return dq, dk, dv
 
 

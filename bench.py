@@ -584,12 +584,11 @@ def aux_localize(fm, torch, dev, stream, hbm, reps=20):
     work = pairs.sum(dim=(1, 2, 3)).double()
     out["kv_chunk_pairs"].update(chunks_pruned=int((pairs == 0).sum().item()), chunks=int(pairs.numel()),
                                  rank_work_max_over_mean=round(float(work.max() / work.mean()), 4))
-    # sparsity-aware assignment: per-chunk work from the same passes, longest-first vs dual-chunk
+    # sparsity-aware assignment: per-chunk work from the same passes; dual-chunk, longest-first and
+    # refined assignments against the bound set by the chunk granularity
     from mask_aware_flash_b200 import cp_balance as cb
     cost = cb.chunk_costs(fm, vt, chunk)
-    out["balance"] = {"ranks": R, "chunks_per_rank": 2,
-                      "dual_chunk_max_over_mean": round(cb.imbalance(cost, cb.dual_chunk(nch)), 4),
-                      "longest_first_max_over_mean": round(cb.imbalance(cost, cb.assign_longest_first(cost, R, 2)), 4)}
+    out["balance"] = cb.balance_report(cost, R, 2)
     return out
 
 

@@ -11,8 +11,11 @@ counts; an assignment is then scored by max / mean work over the ranks.
 `assign_longest_first` is longest-processing-time-first with a fixed number of
 chunks per rank (every rank holds the same number of tokens, as under the
 dual-chunk assignment): chunks in descending cost, each to the currently
-lightest rank that still has room (ties: lowest rank).  Chunks of one rank are
-returned in increasing global order, as fm_localize requires.
+lightest rank that still has room (ties: lowest rank).  `refine_by_swaps`
+then exchanges chunks between the heaviest rank and another one while that
+lowers the maximum (pairwise interchange, a standard local search for
+equal-cardinality partitioning).  Chunks of one rank are returned in
+increasing global order, as fm_localize requires.
 """
 from __future__ import annotations
 
@@ -44,10 +47,64 @@ def assign_longest_first(cost, ranks: int, per_rank: int):
     return [sorted(x) for x in owned]
 
 
+def refine_by_swaps(cost, assignment, max_rounds: int = 10000):
+    """Pairwise-interchange local search on an assignment with equal chunks per rank: while some
+    exchange of one chunk of the heaviest rank with one chunk of another rank lowers the heavier
+    of the two ranks below the current maximum, make the exchange that lowers it most (ties: lowest
+    rank, then lowest chunk ids).  Ranks keep their chunk counts, the maximum work never grows,
+    and the result is returned as sorted chunk lists like the input."""
+    cost = np.asarray(cost, dtype=np.int64)
+    owned = [sorted(int(c) for c in x) for x in assignment]
+    work = [int(cost[x].sum()) if x else 0 for x in owned]
+    for _ in range(max_rounds):
+        hi = max(range(len(owned)), key=lambda r: (work[r], -r))
+        best = None  # (new max of the pair, rank, chunk out of hi, chunk in from rank)
+        for r in range(len(owned)):
+            if r == hi:
+                continue
+            for a in owned[hi]:
+                for b in owned[r]:
+                    d = int(cost[a]) - int(cost[b])  # work moved from hi to r
+                    if d <= 0:
+                        continue
+                    pair_max = max(work[hi] - d, work[r] + d)
+                    if pair_max < work[hi] and (best is None or (pair_max, r, a, b) < best):
+                        best = (pair_max, r, a, b)
+        if best is None:
+            break
+        _, r, a, b = best
+        d = int(cost[a]) - int(cost[b])
+        owned[hi].remove(a)
+        owned[hi].append(b)
+        owned[r].remove(b)
+        owned[r].append(a)
+        work[hi] -= d
+        work[r] += d
+    return [sorted(x) for x in owned]
+
+
 def imbalance(cost, assignment) -> float:
     """max / mean of the per-rank work of an assignment."""
     work = np.array([sum(int(cost[c]) for c in chunks) for chunks in assignment], dtype=np.float64)
     return float(work.max() / work.mean()) if work.mean() > 0 else 1.0
+
+
+def balance_report(cost, ranks: int, per_rank: int) -> dict:
+    """max / mean per-rank work of the dual-chunk, longest-first and refined assignments of
+    `cost` (ranks * per_rank chunks), with the lower bound that no assignment with per_rank
+    chunks per rank can beat: max(mean, the largest chunk plus the per_rank - 1 smallest)."""
+    cost = np.asarray(cost, dtype=np.int64)
+    mean = float(cost.sum()) / ranks
+    lpt = assign_longest_first(cost, ranks, per_rank)
+    srt = np.sort(cost)
+    bound = max(mean, float(srt[-1] + srt[:per_rank - 1].sum()))
+    out = {"ranks": ranks, "chunks_per_rank": per_rank}
+    if per_rank == 2:
+        out["dual_chunk_max_over_mean"] = round(imbalance(cost, dual_chunk(len(cost))), 4)
+    out["longest_first_max_over_mean"] = round(imbalance(cost, lpt), 4)
+    out["refined_max_over_mean"] = round(imbalance(cost, refine_by_swaps(cost, lpt)), 4)
+    out["lower_bound_max_over_mean"] = round(bound / mean, 4) if mean > 0 else 1.0
+    return out
 
 
 def chunk_costs(fm, vecs, chunk_len: int):

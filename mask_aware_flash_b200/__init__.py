@@ -117,6 +117,14 @@ def _vecs(vecs):
     return VecArray(*[None if v is None else v.data_ptr() for v in vecs])
 
 
+def _first_vector(vecs, what):
+    """The first non-None vector (it gives the shape); all None is an invalid call."""
+    ref = next((v for v in vecs if v is not None), None)
+    if ref is None:
+        raise FmError(FM_ERR_INVALID_ARG, f"{what}: at least one vector must be given (it sets the shape)")
+    return ref
+
+
 class MaskMeta:
     """Tile metadata (views into an owned workspace tensor)."""
 
@@ -151,7 +159,7 @@ def fm_mask_meta_workspace_bytes(B, Hm, n_q, n_k) -> int:
 
 def fm_build_mask_meta(lts, lte, uts, ute, n_q: int, stream=None) -> MaskMeta:
     """Vectors: int32 CUDA tensors [B, Hm, n_k] (or None = canonical empty)."""
-    ref = next(v for v in (lts, lte, uts, ute) if v is not None)
+    ref = _first_vector((lts, lte, uts, ute), "fm_build_mask_meta")
     B, Hm, n_k = ref.shape
     d = MaskDesc(B, Hm, n_q, n_k, TILE, TILE)
     nbytes = lib().fm_mask_meta_workspace_bytes(ctypes.byref(d))
@@ -171,8 +179,9 @@ def fm_localize(vecs, chunk_start, chunk_len, out=None, stream=None):
     cs = np.ascontiguousarray(np.asarray(chunk_start, dtype=np.int32))
     cl = np.ascontiguousarray(np.asarray(chunk_len, dtype=np.int32))
     R, C = cs.shape
-    B, Hm, N = vecs[0].shape
-    outs = out if out is not None else [torch.empty((R, B, Hm, N), dtype=torch.int32, device=vecs[0].device)
+    ref = _first_vector(vecs, "fm_localize")
+    B, Hm, N = ref.shape
+    outs = out if out is not None else [torch.empty((R, B, Hm, N), dtype=torch.int32, device=ref.device)
                                         for _ in range(4)]
     _check(lib().fm_localize(B, Hm, N, _vecs(vecs), R, C, cs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                              cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _vecs(outs), _stream(stream)),
@@ -184,7 +193,7 @@ def fm_kv_chunk_pairs(loc_vecs, n_loc, chunk_len: int, out=None, stream=None):
     """loc_vecs: 4 int32 CUDA tensors [R, B, Hm, N] (fm_localize's output; None = canonical empty);
     n_loc: R host ints.  Returns int64 [R, B, Hm, ceil(N / chunk_len)] unmasked-pair counts per KV chunk."""
     import numpy as np
-    ref = next(v for v in loc_vecs if v is not None)
+    ref = _first_vector(loc_vecs, "fm_kv_chunk_pairs")
     R, B, Hm, N = ref.shape
     nl = np.ascontiguousarray(np.asarray(n_loc, dtype=np.int32))
     if nl.shape != (R,):

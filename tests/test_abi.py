@@ -207,3 +207,12 @@ def test_varlen_binding_rejects_non_int32():
         fm.fm_varlen_mask(torch.zeros(3, dtype=torch.int64), 10)
     with pytest.raises(fm.FmError):
         fm.fm_varlen_mask(torch.zeros((2, 2), dtype=torch.int32), 10)
+
+
+def test_binding_needs_one_vector_for_the_shape():
+    with pytest.raises(fm.FmError):
+        fm.fm_build_mask_meta(None, None, None, None, n_q=128)
+    with pytest.raises(fm.FmError):
+        fm.fm_kv_chunk_pairs([None] * 4, [64], 64)
+    with pytest.raises(fm.FmError):
+        fm.fm_localize([None] * 4, [[0]], [[64]])

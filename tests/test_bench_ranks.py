@@ -67,3 +67,25 @@ def test_reference_arm_only_on_rank0():
                         "--warmup", "0"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("config", ["n8192", "n32768", "n131072"])
+def test_bench_unmasked_pairs_match_oracle(config):
+    """The U behind every effective-TFLOP/s figure of the bench (4·D·U·H forward, 10·D·U·H
+    backward): the bench's interval count equals the oracle's count for each batch row of each
+    mask of the workload."""
+    import oracle
+    wl = bench.workload(config, 0)
+    n = wl["n"]
+    for name, rows in wl["masks"]:
+        got = bench.unmasked_pairs(rows, n)
+        want = [oracle.count_unmasked(n, n, *s.vectors()) for s in rows]
+        assert got == want, name
+
+
+def test_bench_unmasked_pairs_match_dense_small():
+    import oracle
+    import synth
+    n = 384
+    rows = [synth.make_family(f, n, 3) for f in synth.SWEEP_FAMILIES]
+    assert bench.unmasked_pairs(rows, n) == [oracle.count_unmasked_dense(n, n, *s.vectors()) for s in rows]

@@ -2,7 +2,8 @@
 (world size 2): every rank takes the same collective steps, the reported
 device time is the maximum over ranks, the whole-job value counts every
 rank's replica, each rank draws its own seeded workload of the same shape,
-and the reference arm runs on rank 0 only."""
+and the reference arm runs on rank 0 only.  Also on CPU: the unmasked-pair
+counts behind the bench's FLOP figures equal the oracle's."""
 import json
 import os
 import socket

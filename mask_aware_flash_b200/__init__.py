@@ -117,6 +117,35 @@ def _vecs(vecs):
     return VecArray(*[None if v is None else v.data_ptr() for v in vecs])
 
 
+def _check_tensors(what, device, items):
+    """The C ABI sees raw pointers only: reject here host tensors, tensors of another device,
+    non-contiguous views and wrong element types or shapes.  items: (name, tensor or None,
+    dtype or None, shape or None); None entries are skipped (NULL vectors are legal)."""
+    for name, t, dtype, shape in items:
+        if t is None:
+            continue
+        if not t.is_cuda or t.device != device:
+            raise FmError(FM_ERR_INVALID_ARG, f"{what}: {name} must be a CUDA tensor on {device}")
+        if not t.is_contiguous():
+            raise FmError(FM_ERR_INVALID_ARG, f"{what}: {name} must be contiguous")
+        if dtype is not None and t.dtype != dtype:
+            raise FmError(FM_ERR_INVALID_ARG, f"{what}: {name} must be {dtype}, not {t.dtype}")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise FmError(FM_ERR_INVALID_ARG, f"{what}: {name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+
+
+def _check_qkv(what, q, k, v):
+    """q [B, n_q, H, D] and k, v [B, n_k, H_kv, D] of one element type (bf16 or fp32)."""
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise FmError(FM_ERR_INVALID_ARG, f"{what}: q, k, v must be 4-D [B, n, heads, D]")
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise FmError(FM_ERR_INVALID_ARG, f"{what}: q must be bfloat16 or float32, not {q.dtype}")
+    B, _, _, D = q.shape
+    kv_shape = (B, k.shape[1], k.shape[2], D)
+    _check_tensors(what, q.device, [("q", q, None, None), ("k", k, q.dtype, kv_shape), ("v", v, q.dtype, kv_shape)])
+    return tuple(q.shape), kv_shape
+
+
 def _first_vector(vecs, what):
     """The first non-None vector (it gives the shape); all None is an invalid call."""
     ref = next((v for v in vecs if v is not None), None)
@@ -160,7 +189,11 @@ def fm_mask_meta_workspace_bytes(B, Hm, n_q, n_k) -> int:
 def fm_build_mask_meta(lts, lte, uts, ute, n_q: int, stream=None) -> MaskMeta:
     """Vectors: int32 CUDA tensors [B, Hm, n_k] (or None = canonical empty)."""
     ref = _first_vector((lts, lte, uts, ute), "fm_build_mask_meta")
+    if ref.dim() != 3:
+        raise FmError(FM_ERR_INVALID_ARG, "fm_build_mask_meta: vectors must be [B, Hm, n_k]")
     B, Hm, n_k = ref.shape
+    _check_tensors("fm_build_mask_meta", ref.device,
+                   [(nm, t, torch.int32, ref.shape) for nm, t in zip(("lts", "lte", "uts", "ute"), (lts, lte, uts, ute))])
     d = MaskDesc(B, Hm, n_q, n_k, TILE, TILE)
     nbytes = lib().fm_mask_meta_workspace_bytes(ctypes.byref(d))
     if nbytes == 0:
@@ -180,9 +213,14 @@ def fm_localize(vecs, chunk_start, chunk_len, out=None, stream=None):
     cl = np.ascontiguousarray(np.asarray(chunk_len, dtype=np.int32))
     R, C = cs.shape
     ref = _first_vector(vecs, "fm_localize")
+    if ref.dim() != 3:
+        raise FmError(FM_ERR_INVALID_ARG, "fm_localize: vectors must be [B, Hm, N]")
     B, Hm, N = ref.shape
     outs = out if out is not None else [torch.empty((R, B, Hm, N), dtype=torch.int32, device=ref.device)
                                         for _ in range(4)]
+    _check_tensors("fm_localize", ref.device,
+                   [(f"vecs[{c}]", vecs[c], torch.int32, ref.shape) for c in range(4)] +
+                   [(f"out[{c}]", outs[c], torch.int32, (R, B, Hm, N)) for c in range(4)])
     _check(lib().fm_localize(B, Hm, N, _vecs(vecs), R, C, cs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                              cl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _vecs(outs), _stream(stream)),
            "fm_localize")
@@ -194,12 +232,19 @@ def fm_kv_chunk_pairs(loc_vecs, n_loc, chunk_len: int, out=None, stream=None):
     n_loc: R host ints.  Returns int64 [R, B, Hm, ceil(N / chunk_len)] unmasked-pair counts per KV chunk."""
     import numpy as np
     ref = _first_vector(loc_vecs, "fm_kv_chunk_pairs")
+    if ref.dim() != 4:
+        raise FmError(FM_ERR_INVALID_ARG, "fm_kv_chunk_pairs: vectors must be [R, B, Hm, N]")
     R, B, Hm, N = ref.shape
     nl = np.ascontiguousarray(np.asarray(n_loc, dtype=np.int32))
     if nl.shape != (R,):
         raise FmError(FM_ERR_INVALID_ARG, "fm_kv_chunk_pairs: n_loc must hold one row count per rank")
+    if int(chunk_len) < 1:
+        raise FmError(FM_ERR_INVALID_ARG, "fm_kv_chunk_pairs: chunk_len must be >= 1")
     if out is None:
         out = torch.empty((R, B, Hm, -(-N // chunk_len)), dtype=torch.int64, device=ref.device)
+    _check_tensors("fm_kv_chunk_pairs", ref.device,
+                   [(f"loc_vecs[{c}]", loc_vecs[c], torch.int32, ref.shape) for c in range(4)] +
+                   [("out", out, torch.int64, (R, B, Hm, -(-N // chunk_len)))])
     _check(lib().fm_kv_chunk_pairs(B, Hm, N, R, _vecs(loc_vecs), nl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                                    int(chunk_len), _ptr(out), _stream(stream)), "fm_kv_chunk_pairs")
     return out
@@ -212,6 +257,9 @@ def fm_varlen_mask(cu_seqlens, N: int, causal: bool = True, out=None, stream=Non
         raise FmError(FM_ERR_INVALID_ARG, "fm_varlen_mask: cu_seqlens must be a contiguous int32 vector")
     if out is None:
         out = [torch.empty((1, 1, N), dtype=torch.int32, device=cu_seqlens.device) for _ in range(4)]
+    _check_tensors("fm_varlen_mask", cu_seqlens.device,
+                   [("cu_seqlens", cu_seqlens, None, None)] + [(f"out[{c}]", out[c], torch.int32, (1, 1, N))
+                                                             for c in range(4)])
     _check(lib().fm_varlen_mask(_ptr(cu_seqlens), cu_seqlens.numel() - 1, int(N), 1 if causal else 0,
                                 *[_ptr(x) for x in out], _stream(stream)), "fm_varlen_mask")
     return out
@@ -227,11 +275,15 @@ def _args(q, k, v, scale, deterministic=False) -> AttnArgs:
 def fm_attn_fwd(q, k, v, meta: MaskMeta, vecs, scale, o=None, lse=None, stream=None):
     """q [B, n_q, H, D], k/v [B, n_k, H_kv, D] CUDA tensors (bf16, or fp32 with D=64; H % H_kv == 0)
     -> o (same dtype), lse [B, H, n_q] fp32."""
-    B, n_q, H, D = q.shape
+    q_shape, _ = _check_qkv("fm_attn_fwd", q, k, v)
+    B, n_q, H, D = q_shape
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
+    d = meta.desc
+    _check_tensors("fm_attn_fwd", q.device, [("o", o, q.dtype, q_shape), ("lse", lse, torch.float32, (B, H, n_q))] +
+                   [(f"vecs[{c}]", vecs[c], torch.int32, (d.B, d.Hm, d.n_k)) for c in range(4)])
     a = _args(q, k, v, scale)
     _check(lib().fm_attn_fwd(ctypes.byref(a), ctypes.byref(meta.c), _vecs(vecs), _ptr(o), _ptr(lse),
                              _stream(stream)), "fm_attn_fwd")
@@ -247,6 +299,8 @@ def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=No
                 stream=None, deterministic=False):
     """Gradients (dtype of q) of the masked attention; ws: optional uint8 CUDA workspace.
     deterministic: add the key tiles' dQ contributions in a fixed order (bitwise repeatable dQ)."""
+    q_shape, kv_shape = _check_qkv("fm_attn_bwd", q, k, v)
+    B, n_q, H, D = q_shape
     a = _args(q, k, v, scale, deterministic)
     nbytes = lib().fm_attn_bwd_workspace_bytes(ctypes.byref(a))
     if ws is None:
@@ -254,6 +308,12 @@ def fm_attn_bwd(q, k, v, o, lse, do, meta: MaskMeta, vecs, scale, dq=None, dk=No
     dq = torch.empty_like(q) if dq is None else dq  # dk, dv: the shape of k, v ([B, n_k, H_kv, D])
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    d = meta.desc
+    _check_tensors("fm_attn_bwd", q.device,
+                   [("o", o, q.dtype, q_shape), ("lse", lse, torch.float32, (B, H, n_q)), ("do", do, q.dtype, q_shape),
+                    ("dq", dq, q.dtype, q_shape), ("dk", dk, q.dtype, kv_shape), ("dv", dv, q.dtype, kv_shape),
+                    ("ws", ws, None, None)] +
+                   [(f"vecs[{c}]", vecs[c], torch.int32, (d.B, d.Hm, d.n_k)) for c in range(4)])
     _check(lib().fm_attn_bwd(ctypes.byref(a), ctypes.byref(meta.c), _vecs(vecs), _ptr(o), _ptr(lse), _ptr(do),
                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "fm_attn_bwd")

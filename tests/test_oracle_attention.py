@@ -181,3 +181,41 @@ def test_per_head_vectors():
     c1 = oracle.attention_head(q, k, v, [None] * 4, 0, 1, 0.3)
     np.testing.assert_array_equal(r0["o"], c0["o"])
     np.testing.assert_array_equal(r1["o"], c1["o"])
+
+
+@pytest.mark.parametrize("family", ["causal_document", "global_sliding"])
+def test_grouped_query_reading_vs_torch_sdpa(family):
+    """Grouped-query attention as the GPU tests check it: the oracle run on K / V repeated to H
+    heads (query head h reads K/V head h // (H / H_kv)), dK / dV of a K/V head summed over its query
+    heads, equals PyTorch's fp64 SDPA with enable_gqa=True + autograd."""
+    n, H, H_kv, D = 64, 6, 2, 16
+    g = H // H_kv
+    spec = synth.make_family(family, n, 31)
+    q, _, _, do = _inputs(1, n, n, H, D, 8)
+    _, k, v, _ = _inputs(1, n, n, H_kv, D, 9)
+    vecs = [x[None, None, :] for x in spec.vectors()]
+    allowed = ~oracle.dense_mask(n, n, *spec.vectors())
+    assert allowed.any(axis=1).all()  # no dead rows, so SDPA stays finite everywhere
+    scale = 1.0 / math.sqrt(D)
+    k_rep, v_rep = np.repeat(k, g, axis=2), np.repeat(v, g, axis=2)
+    dk = np.zeros((n, H_kv, D))
+    dv = np.zeros((n, H_kv, D))
+    rows = []
+    for h in range(H):
+        r = _full(q, k_rep, v_rep, do, vecs, 0, h, scale)
+        rows.append(r)
+        dk[:, h // g] += r["dk"]
+        dv[:, h // g] += r["dv"]
+    Q = torch.tensor(q[0].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)  # [H, n, D]
+    K = torch.tensor(k[0].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)  # [H_kv, n, D]
+    V = torch.tensor(v[0].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+    O = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None],
+                                                         attn_mask=torch.tensor(allowed)[None, None], scale=scale,
+                                                         enable_gqa=True)[0]
+    (O * torch.tensor(do[0].transpose(1, 0, 2), dtype=torch.float64)).sum().backward()
+    for h in range(H):
+        np.testing.assert_allclose(rows[h]["o"], O[h].detach().numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(rows[h]["dq"], Q.grad[h].numpy(), rtol=1e-9, atol=1e-11)
+    for hk in range(H_kv):
+        np.testing.assert_allclose(dk[:, hk], K.grad[hk].numpy(), rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(dv[:, hk], V.grad[hk].numpy(), rtol=1e-9, atol=1e-11)

@@ -219,3 +219,29 @@ def test_grouped_query_reading_vs_torch_sdpa(family):
     for hk in range(H_kv):
         np.testing.assert_allclose(dk[:, hk], K.grad[hk].numpy(), rtol=1e-9, atol=1e-11)
         np.testing.assert_allclose(dv[:, hk], V.grad[hk].numpy(), rtol=1e-9, atol=1e-11)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_packing_vs_torch_sdpa_per_sequence(causal):
+    """A packed batch under the varlen vectors: every sequence's rows of O / dQ and keys of dK / dV
+    equal PyTorch's fp64 SDPA (+ autograd) on that sequence alone (causal or unmasked); padding
+    rows are dead (LSE = -inf) and padding keys get zero gradients."""
+    cu = [0, 13, 40, 40, 57]
+    N, H, D = 64, 1, 8
+    q, k, v, do = _inputs(1, N, N, H, D, 12)
+    vecs = [x[None, None, :] for x in oracle.varlen_vectors(cu, N, causal)]
+    r = _full(q, k, v, do, vecs, 0, 0, 0.3)
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        if a == b:
+            continue
+        Q, K, V = (torch.tensor(x[0, a:b, 0], dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+        O = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None], is_causal=causal,
+                                                             scale=0.3)[0]
+        (O * torch.tensor(do[0, a:b, 0], dtype=torch.float64)).sum().backward()
+        np.testing.assert_allclose(r["o"][a:b], O.detach().numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(r["dq"][a:b], Q.grad.numpy(), rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(r["dk"][a:b], K.grad.numpy(), rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(r["dv"][a:b], V.grad.numpy(), rtol=1e-9, atol=1e-11)
+    assert np.all(np.isneginf(r["lse"][cu[-1]:]))
+    assert np.all(r["dk"][cu[-1]:] == 0) and np.all(r["dv"][cu[-1]:] == 0)

@@ -263,15 +263,18 @@ static double dot_f(const float* a, const float* b, int D) {
   return s;
 }
 
-// one row: LSE_i and O_i (O written to o[D])
-static double row_forward(const Problem& p, const Vecs& vv, int64_t i, double* o) {
+// One row: its scores s_ij = scale q_i.k_j on the unmasked keys are formed once
+// into s[0, n_k) (entries of masked keys are left untouched and never read);
+// then LSE_i and O_i (O written to o[D]) by the three passes of the definition:
+// the maximum, the sum of exp(s - m), and the weighted sum of the V rows.
+static double row_forward(const Problem& p, const Vecs& vv, int64_t i, double* s, double* o) {
   const int D = p.D;
   double m = -std::numeric_limits<double>::infinity();
   bool any = false;
   for (int64_t j = 0; j < p.n_k; ++j) {
     if (vv.masked(i, j)) continue;
-    double s = p.scale * dot_f(p.Q(i), p.K(j), D);
-    if (!any || s > m) m = s;
+    s[j] = p.scale * dot_f(p.Q(i), p.K(j), D);
+    if (!any || s[j] > m) m = s[j];
     any = true;
   }
   for (int d = 0; d < D; ++d) o[d] = 0.0;
@@ -279,12 +282,12 @@ static double row_forward(const Problem& p, const Vecs& vv, int64_t i, double* o
   double l = 0.0;
   for (int64_t j = 0; j < p.n_k; ++j) {
     if (vv.masked(i, j)) continue;
-    l += std::exp(p.scale * dot_f(p.Q(i), p.K(j), D) - m);
+    l += std::exp(s[j] - m);
   }
   double lse = m + std::log(l);
   for (int64_t j = 0; j < p.n_k; ++j) {
     if (vv.masked(i, j)) continue;
-    double pij = std::exp(p.scale * dot_f(p.Q(i), p.K(j), D) - lse);
+    double pij = std::exp(s[j] - lse);
     const float* vj = p.V(j);
     for (int d = 0; d < D; ++d) o[d] += pij * (double)vj[d];
   }
@@ -306,40 +309,46 @@ int orc_attention_head(int32_t B, int32_t H, int32_t Hm, int32_t n_q, int32_t n_
   if (nthreads > 0) omp_set_num_threads(nthreads);
 #endif
   // sampled rows: O, LSE, dQ
-#pragma omp parallel for schedule(dynamic, 1)
-  for (int32_t r = 0; r < n_rows; ++r) {
-    const int64_t i = rows[r];
-    std::vector<double> o(D);
-    double lse = row_forward(p, vv, i, o.data());
-    for (int d = 0; d < D; ++d) o_out[(int64_t)r * D + d] = o[d];
-    lse_out[r] = lse;
-    if (dq_out) {
-      std::vector<double> dq(D, 0.0);
-      if (std::isfinite(lse)) {
-        double Di = 0.0;
-        for (int d = 0; d < D; ++d) Di += (double)p.dO(i)[d] * o[d];
-        for (int64_t j = 0; j < n_k; ++j) {
-          if (vv.masked(i, j)) continue;
-          double pij = std::exp(scale * dot_f(p.Q(i), p.K(j), D) - lse);
-          double dsij = pij * (dot_f(p.dO(i), p.V(j), D) - Di);
-          const float* kj = p.K(j);
-          for (int d = 0; d < D; ++d) dq[d] += scale * dsij * (double)kj[d];
+#pragma omp parallel
+  {
+    std::vector<double> s(n_k), o(D), dq(D);
+#pragma omp for schedule(dynamic, 1)
+    for (int32_t r = 0; r < n_rows; ++r) {
+      const int64_t i = rows[r];
+      double lse = row_forward(p, vv, i, s.data(), o.data());
+      for (int d = 0; d < D; ++d) o_out[(int64_t)r * D + d] = o[d];
+      lse_out[r] = lse;
+      if (dq_out) {
+        for (int d = 0; d < D; ++d) dq[d] = 0.0;
+        if (std::isfinite(lse)) {
+          double Di = 0.0;
+          for (int d = 0; d < D; ++d) Di += (double)p.dO(i)[d] * o[d];
+          for (int64_t j = 0; j < n_k; ++j) {
+            if (vv.masked(i, j)) continue;
+            double pij = std::exp(s[j] - lse);
+            double dsij = pij * (dot_f(p.dO(i), p.V(j), D) - Di);
+            const float* kj = p.K(j);
+            for (int d = 0; d < D; ++d) dq[d] += scale * dsij * (double)kj[d];
+          }
         }
+        for (int d = 0; d < D; ++d) dq_out[(int64_t)r * D + d] = dq[d];
       }
-      for (int d = 0; d < D; ++d) dq_out[(int64_t)r * D + d] = dq[d];
     }
   }
   if (n_cols <= 0) return 0;
   // all-rows statistics for the column outputs: LSE_i and D_i
   std::vector<double> lse_all(n_q), D_all(n_q);
-#pragma omp parallel for schedule(dynamic, 16)
-  for (int64_t i = 0; i < n_q; ++i) {
-    std::vector<double> o(D);
-    double lse = row_forward(p, vv, i, o.data());
-    lse_all[i] = lse;
-    double Di = 0.0;
-    for (int d = 0; d < D; ++d) Di += (double)p.dO(i)[d] * o[d];
-    D_all[i] = Di;
+#pragma omp parallel
+  {
+    std::vector<double> s(n_k), o(D);
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t i = 0; i < n_q; ++i) {
+      double lse = row_forward(p, vv, i, s.data(), o.data());
+      lse_all[i] = lse;
+      double Di = 0.0;
+      for (int d = 0; d < D; ++d) Di += (double)p.dO(i)[d] * o[d];
+      D_all[i] = Di;
+    }
   }
 #pragma omp parallel for schedule(dynamic, 1)
   for (int32_t c = 0; c < n_cols; ++c) {

@@ -272,9 +272,10 @@ fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int
  *     FM_BWD_NOALLOC_SCRATCH_BYTES (for D = 128 about 64K query rows in total,
  *     B * H * n_q); larger problems are rejected with FM_ERR_WORKSPACE before
  *     any launch.
- *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *   - Every call looks up the array's address on the current device (a
+ *     symbol lookup, nothing allocated), so the address never goes stale; the
+ *     first lookup on a device may load the library's device code, so make
+ *     the first call before any stream capture.
  *   - Every call on a device shares the one array; it keeps the last call's
  *     contents and each call clears what must start at zero.  Calls whose
  *     kernels overlap on the GPU (different streams, no ordering between

@@ -9,12 +9,12 @@
 
 namespace fm {
 
-// Latched device-side error (FM_ERR_DEVICE_TIMEOUT << 16 | site), one per device.
+// Latched device-side error (FM_ERR_DEVICE_TIMEOUT << 16 | site), one per device, and the slot into
+// which fm_get_device_status moves it (read and cleared in one atomic exchange).
 __device__ int g_fm_status;
+__device__ int g_fm_status_taken;
 
 namespace {
-constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {};
 std::mutex g_mu;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -36,16 +36,12 @@ EncodeTiledFn get_encode() {
 }
 }  // namespace
 
+// Device address of the status word on the current device, looked up on every call (a cached
+// address would go stale after cudaDeviceReset or a new primary context).
 int* device_status_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_fm_status) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  return g_status_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_fm_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
 
 // 4-D map over a [B, n, H, D] bf16 tensor: dims (D, H, n, B), box (64, 1, box_rows, 1),
@@ -94,6 +90,11 @@ __global__ void selftest_wait_kernel(int* status) {
   if (threadIdx.x == 0 && !mbar_wait(smem_u32(&bar), 0, &abort_flag)) record_failure(status, &abort_flag, 0x7E57);
 }
 
+
+// Moves the status word into `taken` and clears it in one atomic exchange, so a failure that a
+// kernel on another stream latches concurrently is either returned now or kept for the next read.
+__global__ void take_status_kernel(int* status, int* taken) { *taken = atomicExch(status, 0); }
+
 }  // namespace fm
 
 extern "C" {
@@ -119,11 +120,14 @@ const char* fm_status_string(fm_status s) {
 
 fm_status fm_get_device_status(fm_stream_t stream) {
   int* p = fm::device_status_ptr();
-  if (!p) return FM_ERR_CUDA;
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FM_ERR_CUDA;
-  int v = 0, zero = 0;
-  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FM_ERR_CUDA;
-  if (v != 0 && cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FM_ERR_CUDA;
+  void* taken = nullptr;
+  if (!p || cudaGetSymbolAddress(&taken, fm::g_fm_status_taken) != cudaSuccess) return FM_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  fm::take_status_kernel<<<1, 1, 0, s>>>(p, static_cast<int*>(taken));
+  int v = 0;
+  if (cudaGetLastError() != cudaSuccess || cudaMemcpyAsync(&v, taken, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return FM_ERR_CUDA;
   return v == 0 ? FM_OK : static_cast<fm_status>(v >> 16);
 }
 

@@ -22,8 +22,6 @@
 // and the log2-domain LSE (rows padded to whole query tiles) and clears the
 // accumulator; a final kernel scales the accumulator into dQ.  The fp32 path
 // (kind::tf32) transposes its MN-major operands in shared memory (drain warps).
-#include <mutex>
-
 #include "fm_common.cuh"
 
 namespace fm {
@@ -869,20 +867,13 @@ fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int
 static __device__ __align__(256) uint8_t g_bwd_noalloc_scratch[FM_BWD_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
-
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array on the current device.  Looked up on every call (a symbol
+// lookup, no allocation): a cached address would go stale after cudaDeviceReset or a new primary
+// context, and the kernels would then write through it.
 void* noalloc_scratch() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = p;
-  }
-  return g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_bwd_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 }  // namespace
 

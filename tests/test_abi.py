@@ -13,6 +13,11 @@ from mask_aware_flash_b200 import _build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def torch_cuda_present():
+    import torch
+    return torch.cuda.is_available()
+
+
 @pytest.fixture(scope="module")
 def L():
     _build.build()
@@ -216,3 +221,21 @@ def test_binding_needs_one_vector_for_the_shape():
         fm.fm_kv_chunk_pairs([None] * 4, [64], 64)
     with pytest.raises(fm.FmError):
         fm.fm_localize([None] * 4, [[0]], [[64]])
+
+
+@pytest.mark.skipif(torch_cuda_present(), reason="hands made-up device addresses to an entry point that can launch")
+def test_noalloc_rejects_oversize(L):
+    """fm_attn_bwd_noalloc: a problem beyond its fixed scratch fails on the host, before any CUDA call."""
+    L.fm_attn_bwd_noalloc.argtypes = [ctypes.POINTER(fm.AttnArgs), ctypes.POINTER(fm.MaskMetaC), fm.VecArray] + \
+        [ctypes.c_void_p] * 7
+    L.fm_attn_bwd_noalloc.restype = ctypes.c_int
+    D, H = 128, 16
+    n = 8192  # B*H*n_q = 131072 rows of fp32 dQ accumulator: 64 MiB > 32 MiB
+    a = fm.AttnArgs(1, H, n, n, D, 0, 0.1, 0x10000, 0x20000, 0x30000)
+    m = fm.MaskMetaC()
+    m.d = fm.MaskDesc(1, 1, n, n, 128, 128)
+    m.row_count = m.row_entries = m.col_count = m.col_entries = m.tile_minmax = 0x40000
+    m.tile_class = m.fwd_order = m.bwd_order = 0x40000
+    p = [ctypes.c_void_p(0x100000 * (t + 1)) for t in range(6)]
+    rc = L.fm_attn_bwd_noalloc(ctypes.byref(a), ctypes.byref(m), fm.VecArray(None, None, None, None), *p, None)
+    assert rc == fm.FM_ERR_WORKSPACE

@@ -2,18 +2,22 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input:
 for each mask of the workload, the tile metadata pass, the forward and the
-backward; plus one clip-shift-max localization of the batch's vectors to 8
-simulated context-parallel ranks (dual-chunk assignment).
+backward; plus one clip-shift-max localization of the first mask's vectors to
+8 simulated context-parallel ranks (dual-chunk assignment) and their KV-chunk
+pair counts.
 
-Default workload (N=1): n = 8192, B = 2, H = 16, D = 128, bf16, Q/K/V/dO ~ N(0,1),
-masks (a) causal sliding window w = 1024 and (b) causal documents with lengths
-~ U[512, 4096] (seeded per batch row).
+Default workload (N=1): n = 131072, B = 1, H = 16, D = 128, bf16, Q/K/V/dO ~
+N(0,1), the sweep of 12 seeded structured masks (full, causal, sliding window
+2K and 8K, causal and bidirectional documents, prefix-LM, prefix-LM documents,
+share-question, causal blockwise, global + sliding window, random eviction),
+forward and backward timed per mask.  --config n8192 | n32768 select the
+smaller workloads (two masks each).
 
 Metric: effective TFLOP/s counting only unmasked score entries
 (forward 4*D*U, backward 10*D*U per (b, h), U = unmasked (i, j) pairs).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                       [--config n8192|n32768|n131072]
+                       [--config n131072|n32768|n8192] [--masks a,b,...]
 """
 from __future__ import annotations
 
@@ -45,7 +49,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="n8192", choices=["n8192", "n32768", "n131072"])
+    ap.add_argument("--config", default="n131072", choices=["n131072", "n32768", "n8192"])
     ap.add_argument("--masks", default=None, help="comma list of mask names (default: the config's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -66,8 +70,10 @@ def workload(config: str, rank: int, masks_arg=None):
         desc = "n=32768 B=1 H=32 D=128 bf16; masks: prefix-LM, share-question"
     else:
         n, B, H, D = 131072, 1, 16, 128
-        masks = ["causal", "sliding_window_2k"]
-        desc = "n=131072 B=1 H=16 D=128 bf16; masks: causal, causal sliding window 2K"
+        masks = list(synth.SWEEP_FAMILIES)
+        desc = ("n=131072 B=1 H=16 D=128 bf16; 12-mask sweep: full, causal, sliding window 2K, sliding window 8K, "
+                "causal documents, bidirectional documents, prefix-LM, prefix-LM documents, share-question, "
+                "causal blockwise 64, global + sliding window, random eviction")
     if masks_arg:
         masks = masks_arg.split(",")
         desc = desc.split(";")[0] + "; masks: " + ", ".join(masks)
@@ -229,9 +235,11 @@ def traffic_for(kernel: str, config: str):
 
 # ----------------------------------------------------------------------------- CPU oracle baseline
 def cpu_baseline(wl, budget_s=15.0):
-    """The oracle as it stands, on the host cores: forward + dQ for sampled rows of
-    two heads per mask; effective TFLOP/s = 14 * D * (unmasked pairs of the sampled
-    rows) / time."""
+    """The oracle as it stands, on the host cores: sampled query rows of head (0, 0), one mask per
+    call in turn.  For each unmasked pair of those rows the oracle runs the forward (score, O: 4*D
+    FLOPs in the effective count) and the dQ half of the backward (dP, dQ: 4*D of the backward's
+    10*D); it runs no dK / dV column work here, so it is credited 8*D FLOPs per pair, the FLOPs it
+    actually ran."""
     import oracle
     n, B, H, D = wl["n"], wl["B"], wl["H"], wl["D"]
     scale = 1.0 / math.sqrt(D)
@@ -258,11 +266,11 @@ def cpu_baseline(wl, budget_s=15.0):
         t_used += time.perf_counter() - t0
         done_pairs += allowed_rows
         calls += 1
-    flops = 14.0 * D * done_pairs
+    flops = 8.0 * D * done_pairs
     return {"value": flops / t_used / 1e12, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"{calls} oracle calls x {rows_per_call} sampled query rows (forward + dQ, fp64) of head (0,0) "
-                      f"of the workload's masks, {done_pairs} unmasked pairs in {t_used:.1f} s; "
-                      f"effective FLOPs = 14*D*pairs"}
+            "sample": f"{calls} oracle calls x {rows_per_call} sampled query rows (forward + dQ, fp64) of head (0,0), "
+                      f"the workload's masks in turn, {done_pairs} unmasked pairs in {t_used:.1f} s; "
+                      f"effective FLOPs = 8*D*pairs (forward 4*D + the dQ half of the backward 4*D)"}
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -311,8 +319,9 @@ def run_ours(args, rank, world, local_rank):
     loc_starts = [[r * chunk, (nch - 1 - r) * chunk] for r in range(nch // 2)]
     loc_lens = [[chunk, chunk]] * (nch // 2)
     U = [unmasked_pairs(specs, n) for _, specs in wl["masks"]]
-    flops_fwd = sum(4.0 * D * u * H for us in U for u in us)
-    flops_bwd = sum(10.0 * D * u * H for us in U for u in us)
+    fwd_flops_m = [sum(4.0 * D * u * H for u in us) for us in U]
+    bwd_flops_m = [sum(10.0 * D * u * H for u in us) for us in U]
+    flops_fwd, flops_bwd = sum(fwd_flops_m), sum(bwd_flops_m)
 
     stream = torch.cuda.current_stream()
     o = torch.empty_like(q)
@@ -326,9 +335,9 @@ def run_ours(args, rank, world, local_rank):
     nm = len(wl["masks"])
 
     def build_phases(bs):
-        """The step over one buffer set, as an ordered list of phases (kind, callable, kernel
-        launches): localization of the simulated ranks, their KV-chunk pair counts, then metadata,
-        forward and backward per mask."""
+        """The step over one buffer set, as an ordered list of phases (kind, mask index, callable,
+        kernel launches): localization of the simulated ranks, their KV-chunk pair counts, then
+        metadata, forward and backward per mask."""
         bs["last"], bs["state"] = {"meta": [None] * nm}, {}
         last, state, vd = bs["last"], bs["state"], bs["vec"]
 
@@ -338,7 +347,7 @@ def run_ours(args, rank, world, local_rank):
         def p_kv():
             last["pairs"] = fm.fm_kv_chunk_pairs(state["loc"], n_loc, chunk)
 
-        ph = [("localize", p_loc, 1), ("kv_chunk_pairs", p_kv, 1)]
+        ph = [("localize", -1, p_loc, 1), ("kv_chunk_pairs", -1, p_kv, 1)]
         for mi in range(nm):
             def p_meta(mi=mi):
                 last["meta"][mi] = fm.fm_build_mask_meta(*vd[mi], n_q=n)
@@ -349,20 +358,20 @@ def run_ours(args, rank, world, local_rank):
             def p_bwd(mi=mi):
                 fm.fm_attn_bwd(bs["q"], bs["k"], bs["v"], bs["o"], bs["lse"], bs["do"], last["meta"][mi], vd[mi], scale,
                                dq=bs["dq"], dk=bs["dk"], dv=bs["dv"], ws=bws)
-            ph += [("meta", p_meta, 3), ("fwd", p_fwd, 1), ("bwd", p_bwd, 3)]
+            ph += [("meta", mi, p_meta, fm.META_LAUNCHES), ("fwd", mi, p_fwd, 1), ("bwd", mi, p_bwd, fm.BWD_LAUNCHES)]
         return ph
 
     def capture(ph):
         """Each phase in its own CUDA graph (the host cost of the ctypes calls and output allocations
         would otherwise leave the GPU idle between the small kernels); eager launches if capture fails."""
         if args.no_graph:
-            return [fn for _, fn, _ in ph], False
+            return [x[2] for x in ph], False
         try:
             graphs = []
-            for _, fn, _ in ph:
+            for x in ph:
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
-                    fn()
+                    x[2]()
                 graphs.append(g)
             for g in graphs:  # one replay of the whole step before timing
                 g.replay()
@@ -370,17 +379,17 @@ def run_ours(args, rank, world, local_rank):
             return [g.replay for g in graphs], True
         except Exception as exc:  # keep the eager launches (same kernels)
             print(f"bench: graph capture failed ({exc}); timing eager launches", file=sys.stderr)
-            return [fn for _, fn, _ in ph], False
+            return [x[2] for x in ph], False
 
-    bufs = [dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, vec=vec_dev)]
-    phases = build_phases(bufs[0])
-    last = bufs[0]["last"]
-    launches_per_step = sum(x[2] for x in phases)
+    bs0 = dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv, vec=vec_dev)
+    phases = build_phases(bs0)
+    last = bs0["last"]
+    launches_per_step = sum(x[3] for x in phases)
 
     import torch.distributed as dist
     for _ in range(args.warmup):
-        for _, fn, _ in phases:
-            fn()
+        for x in phases:
+            x[2]()
     torch.cuda.synchronize()
     runners, graphs_used = capture(phases)
     if world > 1:
@@ -404,90 +413,24 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     step_ms = [step_ev[s][0].elapsed_time(step_ev[s][-1]) for s in range(args.steps)]
 
-    def phase_ms(kind):
+    def phase_ms(kind, mi=None):
         return sum(step_ev[s][i].elapsed_time(step_ev[s][i + 1]) for s in range(args.steps)
-                   for i, ph in enumerate(phases) if ph[0] == kind)
+                   for i, ph in enumerate(phases) if ph[0] == kind and (mi is None or ph[1] == mi))
 
-    fwd_ms, bwd_ms, meta_ms = phase_ms("fwd"), phase_ms("bwd"), phase_ms("meta")
-    loc_ms, kvc_ms = phase_ms("localize"), phase_ms("kv_chunk_pairs")
-    total_ms = sum(step_ms)
-    total_ms, fwd_ms, bwd_ms = reduce_max([total_ms, fwd_ms, bwd_ms], world, dev)
     steps = args.steps
+    per_mask_ms = [[phase_ms("fwd", mi), phase_ms("bwd", mi), phase_ms("meta", mi)] for mi in range(nm)]
+    meta_ms = phase_ms("meta")
+    loc_ms, kvc_ms = phase_ms("localize"), phase_ms("kv_chunk_pairs")
+    flat = [sum(step_ms)] + [x for row in per_mask_ms for x in row[:2]]
+    flat = reduce_max(flat, world, dev)  # slowest rank, per quantity
+    total_ms = flat[0]
+    per_mask_ms = [[flat[1 + 2 * mi], flat[2 + 2 * mi], per_mask_ms[mi][2]] for mi in range(nm)]
+    fwd_ms = sum(x[0] for x in per_mask_ms)
+    bwd_ms = sum(x[1] for x in per_mask_ms)
     value = job_tflops(world, flops_fwd + flops_bwd, steps, total_ms)
 
-    # End to end through the public API with host buffers: every step copies its inputs host -> device
-    # from pinned memory and its results device -> host.  Two buffer sets are pipelined: the inputs of
-    # step s+1 go up on one copy stream and the results of step s-1 come back on another while step s
-    # computes; events order every reuse of a buffer set.
-    e2e = None
-    if not args.no_e2e:
-        bufs.append({x: torch.empty_like(bufs[0][x]) for x in ("q", "k", "v", "do", "o", "lse", "dq", "dk", "dv")})
-        bufs[1]["vec"] = [[torch.empty_like(t) for t in vs] for vs in vec_dev]
-        run_e2e = [runners, capture(build_phases(bufs[1]))[0]]
-        out_host = [{x: torch.empty_like(bufs[0][x], device="cpu").pin_memory() for x in ("o", "dq", "dk", "dv", "lse")}
-                    for _ in range(2)]
-        h2d = sum(host[x].numel() * 2 for x in host) + sum(t_.numel() * 4 for vs in vec_host for t_ in vs)
-        d2h = 4 * q.numel() * 2 + lse.numel() * 4
-        up, down = torch.cuda.Stream(), torch.cuda.Stream()
-        new_ev = torch.cuda.Event
-        inputs_ready = [new_ev(), new_ev()]
-        compute_done = [new_ev(), new_ev()]
-        outputs_read = [new_ev(), new_ev()]
-
-        def upload(s_):  # inputs of step s_ into buffer set s_ % 2
-            bs = bufs[s_ % 2]
-            with torch.cuda.stream(up):
-                if s_ >= 2:
-                    up.wait_event(compute_done[s_ % 2])  # step s_-2 has finished reading this set
-                for x in ("q", "k", "v", "do"):
-                    bs[x].copy_(host[x], non_blocking=True)
-                for mi, vs in enumerate(vec_host):
-                    for c in range(4):
-                        bs["vec"][mi][c].copy_(vs[c], non_blocking=True)
-                inputs_ready[s_ % 2].record(up)
-
-        def compute(s_):
-            stream.wait_event(inputs_ready[s_ % 2])
-            if s_ >= 2:
-                stream.wait_event(outputs_read[s_ % 2])  # results of step s_-2 are home
-            for run in run_e2e[s_ % 2]:
-                run()
-            compute_done[s_ % 2].record(stream)
-
-        def download(s_):
-            bs, oh = bufs[s_ % 2], out_host[s_ % 2]
-            with torch.cuda.stream(down):
-                down.wait_event(compute_done[s_ % 2])
-                for x in ("o", "dq", "dk", "dv", "lse"):
-                    oh[x].copy_(bs[x], non_blocking=True)
-                outputs_read[s_ % 2].record(down)
-
-        def pipeline(nsteps, e_start=None, e_end=None):
-            torch.cuda.synchronize()
-            if e_start is not None:
-                e_start.record(stream)
-                up.wait_event(e_start)
-                down.wait_event(e_start)
-            upload(0)
-            for s_ in range(nsteps):
-                if s_ + 1 < nsteps:
-                    upload(s_ + 1)
-                compute(s_)
-                download(s_)
-            stream.wait_event(outputs_read[(nsteps - 1) % 2])
-            if e_end is not None:
-                e_end.record(stream)
-            torch.cuda.synchronize()
-
-        pipeline(max(2, args.warmup))
-        if world > 1:
-            dist.barrier()
-        e0, e1 = ev(), ev()
-        pipeline(steps, e0, e1)
-        (te_ms,) = reduce_max([e0.elapsed_time(e1)], world, dev)
-        e2e = {"value": job_tflops(world, flops_fwd + flops_bwd, steps, te_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "note": "inputs of step s+1 uploaded and results of step s-1 downloaded while step s computes"}
+    e2e = None if args.no_e2e else run_e2e(fm, torch, dev, stream, wl, host, vec_host, scale, bws, steps,
+                                             2, world, flops_fwd + flops_bwd)
     assert fm.fm_get_device_status() == 0, "device-side timeout during the bench"
 
     burst, sustained, hbm, src = peaks()
@@ -509,7 +452,7 @@ def run_ours(args, rank, world, local_rank):
     pairs = last["pairs"]
     rank_work = pairs.sum(dim=(1, 2, 3)).double()
     integer_passes = {
-        "meta": dict(bw(meta_bytes, meta_ms, steps * nm), note="minmax + lists + dispatch order, one call per mask"),
+        "meta": dict(bw(meta_bytes, meta_ms, steps * nm), note="one fm_build_mask_meta call per mask"),
         "localize": dict(bw(16 * B * n * (1 + R), loc_ms, steps), ranks=R),
         "kv_chunk_pairs": dict(bw(16 * B * n * R + 8 * pairs.numel(), kvc_ms, steps), ranks=R,
                                chunks_pruned=int((pairs == 0).sum().item()), chunks=int(pairs.numel()),
@@ -518,31 +461,131 @@ def run_ours(args, rank, world, local_rank):
     }
     fwd_tf = flops_fwd * steps / (fwd_ms * 1e-3) / 1e12
     bwd_tf = flops_bwd * steps / (bwd_ms * 1e-3) / 1e12
+    long_step = total_ms / steps > 200.0  # seconds-long loops run under the power cap
+    peak = sustained if (long_step and sustained) else burst
+    peak_name = "sustained" if peak == sustained and long_step else "burst"
+
+    def frac(tf):
+        return {"effective_tflops": round(tf, 2), "frac_of_2250_nominal": round(tf / 2250.0, 4),
+                "frac_of_measured_burst": round(tf / burst, 4),
+                "frac_of_measured_sustained": round(tf / sustained, 4) if sustained else None}
+
+    masks_out = []
+    for mi, (name, _) in enumerate(wl["masks"]):
+        f_ms, b_ms, m_ms = per_mask_ms[mi]
+        masks_out.append({"mask": name, "unmasked_pairs_per_head": U[mi],
+                          "fwd_ms": round(f_ms / steps, 4), "bwd_ms": round(b_ms / steps, 4),
+                          "meta_ms": round(m_ms / steps, 4),
+                          "fwd": frac(fwd_flops_m[mi] * steps / (f_ms * 1e-3) / 1e12),
+                          "bwd": frac(bwd_flops_m[mi] * steps / (b_ms * 1e-3) / 1e12)})
     dominant = "bwd_kernel" if bwd_ms >= fwd_ms else "fwd_kernel"
     ach = bwd_tf if dominant == "bwd_kernel" else fwd_tf
-    peak = burst
-    launches_per_traffic = {"fwd_kernel": B * H * (n // 128), "bwd_kernel": B * H * (n // 128)}
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), seeded masks)",
         "config": dict(workload_config(wl, world),
                        launch="one CUDA graph per phase, replayed" if graphs_used else "eager",
-                       l2="flushed between steps (256 MiB write outside the step events); inputs 256 MiB > L2"),
-        "fwd": {"effective_tflops": round(fwd_tf, 2), "frac_of_measured_burst": round(fwd_tf / burst, 4),
-                "frac_of_2250_nominal": round(fwd_tf / 2250.0, 4), "ms_per_step": round(fwd_ms / steps, 4)},
-        "bwd": {"effective_tflops": round(bwd_tf, 2), "frac_of_measured_burst": round(bwd_tf / burst, 4),
-                "frac_of_2250_nominal": round(bwd_tf / 2250.0, 4), "ms_per_step": round(bwd_ms / steps, 4),
-                "note": "includes the D_i preprocess and dQ convert kernels"},
+                       l2=f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write outside the step events); "
+                          f"inputs {4 * q.numel() * 2 >> 20} MiB > L2"),
+        "fwd": dict(frac(fwd_tf), ms_per_step=round(fwd_ms / steps, 4)),
+        "bwd": dict(frac(bwd_tf), ms_per_step=round(bwd_ms / steps, 4),
+                    note=f"fm_attn_bwd phase: {fm.BWD_LAUNCHES} launches per call"),
+        "per_mask": masks_out,
         "meta_ms_per_step": round(meta_ms / steps, 4),
         "integer_passes": integer_passes,
         "roofline": {"bound": "tensor", "kernel": dominant, "achieved": round(ach, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-                     "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)",
+                     "peak_source": f"{src} bf16 {peak_name} (MEASURED_PEAKS.json)",
                      "traffic": traffic_for(dominant, args.config)},
         "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
     }
     return line, wl
+
+
+def run_e2e(fm, torch, dev, stream, wl, host, vec_host, scale, bws, steps, warmup, world, flops_step):
+    """End to end through the public API (eager calls, the ones a user makes) with host buffers: every
+    step copies its inputs (Q, K, V, dO and every mask's vectors) from pinned host memory to the GPU,
+    and every mask's results (O, LSE, dQ, dK, dV) back to pinned host memory.  Inputs are
+    double-buffered per step (the inputs of step s+1 go up on one copy stream while step s computes)
+    and outputs per mask (the results of mask m come back on another copy stream while mask m+1
+    computes); events order every reuse of a buffer."""
+    n, B, H = wl["n"], wl["B"], wl["H"]
+    nm = len(wl["masks"])
+    ins = [{x: torch.empty_like(host[x], device=dev) for x in host} for _ in range(2)]
+    for s_ in ins:
+        s_["vec"] = [[torch.empty_like(t, device=dev) for t in vs] for vs in vec_host]
+    outs = [{x: torch.empty_like(ins[0]["q"]) for x in ("o", "dq", "dk", "dv")} for _ in range(2)]
+    for o_ in outs:
+        o_["lse"] = torch.empty((B, H, n), dtype=torch.float32, device=dev)
+    out_host = [{x: torch.empty_like(outs[0][x], device="cpu").pin_memory() for x in outs[0]} for _ in range(2)]
+    h2d = sum(host[x].numel() * 2 for x in host) + sum(t_.numel() * 4 for vs in vec_host for t_ in vs)
+    d2h = nm * sum(t_.numel() * t_.element_size() for t_ in outs[0].values())
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    new_ev = torch.cuda.Event
+    inputs_ready, inputs_free = [new_ev(), new_ev()], [new_ev(), new_ev()]
+    mask_done, outputs_read = [new_ev(), new_ev()], [new_ev(), new_ev()]
+
+    def upload(s_):
+        bs = ins[s_ % 2]
+        with torch.cuda.stream(up):
+            if s_ >= 2:
+                up.wait_event(inputs_free[s_ % 2])  # step s_-2 has finished reading this set
+            for x in ("q", "k", "v", "do"):
+                bs[x].copy_(host[x], non_blocking=True)
+            for mi, vs in enumerate(vec_host):
+                for c in range(4):
+                    bs["vec"][mi][c].copy_(vs[c], non_blocking=True)
+            inputs_ready[s_ % 2].record(up)
+
+    def compute_and_download(s_):
+        bs = ins[s_ % 2]
+        stream.wait_event(inputs_ready[s_ % 2])
+        for mi in range(nm):
+            g = s_ * nm + mi
+            ob, oh = outs[g % 2], out_host[g % 2]
+            if g >= 2:
+                stream.wait_event(outputs_read[g % 2])  # results of mask g-2 are home
+            meta = fm.fm_build_mask_meta(*bs["vec"][mi], n_q=n)
+            fm.fm_attn_fwd(bs["q"], bs["k"], bs["v"], meta, bs["vec"][mi], scale, o=ob["o"], lse=ob["lse"])
+            fm.fm_attn_bwd(bs["q"], bs["k"], bs["v"], ob["o"], ob["lse"], bs["do"], meta, bs["vec"][mi], scale,
+                           dq=ob["dq"], dk=ob["dk"], dv=ob["dv"], ws=bws)
+            mask_done[g % 2].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(mask_done[g % 2])
+                for x in ("o", "lse", "dq", "dk", "dv"):
+                    oh[x].copy_(ob[x], non_blocking=True)
+                outputs_read[g % 2].record(down)
+        inputs_free[s_ % 2].record(stream)
+
+    def pipeline(nsteps, e_start=None, e_end=None):
+        torch.cuda.synchronize()
+        if e_start is not None:
+            e_start.record(stream)
+            up.wait_event(e_start)
+            down.wait_event(e_start)
+        upload(0)
+        for s_ in range(nsteps):
+            if s_ + 1 < nsteps:
+                upload(s_ + 1)
+            compute_and_download(s_)
+        stream.wait_event(outputs_read[(nsteps * nm - 1) % 2])
+        stream.wait_event(outputs_read[(nsteps * nm - 2) % 2])
+        if e_end is not None:
+            e_end.record(stream)
+        torch.cuda.synchronize()
+
+    pipeline(warmup)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pipeline(steps, e0, e1)
+    (te_ms,) = reduce_max([e0.elapsed_time(e1)], world, dev)
+    return {"value": job_tflops(world, flops_step, steps, te_ms), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "note": "eager API calls; inputs of step s+1 uploaded while step s computes, every mask's results "
+                    "downloaded while the next mask computes"}
 
 
 def aux_localize(fm, torch, dev, stream, hbm, reps=20):

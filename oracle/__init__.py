@@ -155,13 +155,20 @@ def attention_head(q, k, v, vecs, b, h, scale, rows=None, cols=None, dout=None, 
     vecs: 4 arrays [B, Hm, n_k] (or None = canonical empty).
     rows: query rows to return (O, LSE, and dQ if dout given); cols: key columns
     for dK, dV (needs dout).  Returns a dict of float64 arrays."""
-    q = np.ascontiguousarray(q, np.float32)
-    k = np.ascontiguousarray(k, np.float32)
-    v = np.ascontiguousarray(v, np.float32)
     B, n_q, H, D = q.shape
     n_k = k.shape[1]
-    dd = None if dout is None else np.ascontiguousarray(dout, np.float32)
-    vv = [None if x is None else _i32(x) for x in vecs]
+    if not (0 <= b < B and 0 <= h < H) or Hm not in (1, H):
+        raise ValueError("oracle: bad arguments")
+    # The C++ code reads only head (b, h): hand it that head as contiguous [1, n, 1, D] copies (and
+    # the head's vector rows), so that its key loop walks memory in order.  Same values, same
+    # arithmetic; only the layout of the input changes.
+    hm = 0 if Hm == 1 else h
+    q = np.ascontiguousarray(q[b:b + 1, :, h:h + 1], np.float32)
+    k = np.ascontiguousarray(k[b:b + 1, :, h:h + 1], np.float32)
+    v = np.ascontiguousarray(v[b:b + 1, :, h:h + 1], np.float32)
+    dd = None if dout is None else np.ascontiguousarray(dout[b:b + 1, :, h:h + 1], np.float32)
+    vv = [None if x is None else _i32(np.asarray(x)[b:b + 1, hm:hm + 1]) for x in vecs]
+    B, H, Hm, b, h = 1, 1, 1, 0, 0
     rows = np.arange(n_q, dtype=np.int32) if rows is None else _i32(rows)
     cols = np.zeros(0, np.int32) if cols is None else _i32(cols)
     if cols.size and dd is None:

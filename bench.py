@@ -624,6 +624,7 @@ def aux_localize(fm, torch, dev, stream, hbm, reps=20):
         gbs = nbytes / (us * 1e-6) / 1e9
         out[name] = {"us_per_launch": round(us, 2), "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1),
                      "frac_of_hbm": round(gbs / hbm, 4)}
+    out["meta_hm16_n131072"] = aux_meta(fm, torch, dev, stream, hbm, reps)
     work = pairs.sum(dim=(1, 2, 3)).double()
     out["kv_chunk_pairs"].update(chunks_pruned=int((pairs == 0).sum().item()), chunks=int(pairs.numel()),
                                  rank_work_max_over_mean=round(float(work.max() / work.mean()), 4))
@@ -633,6 +634,37 @@ def aux_localize(fm, torch, dev, stream, hbm, reps=20):
     cost = cb.chunk_costs(fm, vt, chunk)
     out["balance"] = cb.balance_report(cost, R, 2)
     return out
+
+
+def aux_meta(fm, torch, dev, stream, hbm, reps):
+    """The metadata pass batched over mask heads: one fm_build_mask_meta call on 16 per-head masks
+    (the 12 sweep masks and four more seeds of the first four) of n = 131072 keys, [1, 16, n] vectors
+    (32 MiB).  Algorithmic bytes: the vectors read once; min/max, class matrix, both lists, their
+    counts and both dispatch orders written once."""
+    n, Hm = 131072, 16
+    names = list(synth.SWEEP_FAMILIES) + list(synth.SWEEP_FAMILIES[:4])
+    specs = [synth.make_family(nm, n, 6000 + i) for i, nm in enumerate(names[:Hm])]
+    vt = [torch.from_numpy(np.stack([sp.vectors()[c] for sp in specs])[None].copy()).to(dev) for c in range(4)]
+    meta = fm.fm_build_mask_meta(*vt, n_q=n)
+    ws = meta.ws
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fm.fm_build_mask_meta(*vt, n_q=n, ws=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    T = n // 128
+    ent = int(meta.row_count.sum().item() + meta.col_count.sum().item())
+    nbytes = Hm * (16 * n + 32 * T + T * T + 4 * (T + T) + 4 * (T // 2 + T)) + 4 * ent
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"us_per_launch": round(us, 2), "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1),
+            "frac_of_hbm": round(gbs / hbm, 4), "mask_heads": Hm, "launches_per_call": fm.META_LAUNCHES}
 
 
 def run_reference(args):

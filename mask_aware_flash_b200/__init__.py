@@ -27,8 +27,8 @@ _lib = None
 
 FM_OK, FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA, FM_ERR_DEVICE_TIMEOUT = range(6)
 TILE = 128
-META_LAUNCHES = 3  # kernels one fm_build_mask_meta call launches
-BWD_LAUNCHES = 3   # kernels one fm_attn_bwd call launches (one more with deterministic=True)
+META_LAUNCHES = 2  # kernels one fm_build_mask_meta call launches
+BWD_LAUNCHES = 2   # kernels one fm_attn_bwd call launches (one more with deterministic=True)
 
 
 class FmError(RuntimeError):
@@ -188,8 +188,9 @@ def fm_mask_meta_workspace_bytes(B, Hm, n_q, n_k) -> int:
     return int(lib().fm_mask_meta_workspace_bytes(ctypes.byref(d)))
 
 
-def fm_build_mask_meta(lts, lte, uts, ute, n_q: int, stream=None) -> MaskMeta:
-    """Vectors: int32 CUDA tensors [B, Hm, n_k] (or None = canonical empty)."""
+def fm_build_mask_meta(lts, lte, uts, ute, n_q: int, stream=None, ws=None) -> MaskMeta:
+    """Vectors: int32 CUDA tensors [B, Hm, n_k] (or None = canonical empty).  ws: optional uint8 CUDA
+    workspace of at least fm_mask_meta_workspace_bytes (allocated here when None)."""
     ref = _first_vector((lts, lte, uts, ute), "fm_build_mask_meta")
     if ref.dim() != 3:
         raise FmError(FM_ERR_INVALID_ARG, "fm_build_mask_meta: vectors must be [B, Hm, n_k]")
@@ -200,7 +201,11 @@ def fm_build_mask_meta(lts, lte, uts, ute, n_q: int, stream=None) -> MaskMeta:
     nbytes = lib().fm_mask_meta_workspace_bytes(ctypes.byref(d))
     if nbytes == 0:
         raise FmError(FM_ERR_INVALID_ARG, "fm_mask_meta_workspace_bytes")
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=ref.device)
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=ref.device)
+    _check_tensors("fm_build_mask_meta", ref.device, [("ws", ws, torch.uint8, None)])
+    if ws.numel() < nbytes:
+        raise FmError(FM_ERR_WORKSPACE, "fm_build_mask_meta: workspace too small")
     c = MaskMetaC()
     _check(lib().fm_build_mask_meta(ctypes.byref(d), _ptr(lts), _ptr(lte), _ptr(uts), _ptr(ute), _ptr(ws), nbytes,
                                     ctypes.byref(c), _stream(stream)), "fm_build_mask_meta")

@@ -575,6 +575,417 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Head dimension 256 (bf16).  One 128-row query tile per CTA: S (128 fp32 columns) is double
+// buffered in TMEM next to O (256 columns), S0 | S1 | O = 512 columns.  Q takes 64 KiB of shared
+// memory, so K and V stream through two-slot rings of 64-key halves (32 KiB each): the S product
+// of a 128-key tile is two N = 64 UMMA groups (one per K half), its PV product two K = 64 groups
+// (one per V half, P read from TMEM).  Warp 4 loads Q, K and the mask slices, warp 5 loads V,
+// warp 6 issues the MMAs in the order S(0), S(1), PV(0), S(2), PV(1), S(3), ..., so S(e+1) runs
+// while the softmax of tile e does; warps 0-3 are the softmax (one thread per row), with the same
+// interval test, online softmax and epilogue as the two-tile kernel.
+// ---------------------------------------------------------------------------
+constexpr int kFwd256Threads = 224;
+constexpr int kHalf = 64;  // keys per K / V half tile
+
+struct Fwd256Smem {
+  static constexpr int kQ = 0;                        // 4 atom columns x 128 rows x 128 B
+  static constexpr int kHalfBytes = kHalf * 256 * 2;  // 32 KiB: 4 atom columns x 64 rows x 128 B
+  static constexpr int kK = kQ + 128 * 256 * 2;       // K ring, 2 halves
+  static constexpr int kV = kK + 2 * kHalfBytes;      // V ring, 2 halves
+  static constexpr int kMask = kV + 2 * kHalfBytes;   // [2 buffers][4 vectors][128] int32
+  static constexpr int kList = kMask + 2 * 4 * kTile * 4;
+  static constexpr int kBar = kList + kMaxList * 2;
+  enum { Q_FULL, K_FULL0, K_FULL1, K_EMPTY0, K_EMPTY1, V_FULL0, V_FULL1, V_EMPTY0, V_EMPTY1, S_FULL0, S_FULL1,
+         P_HALF0, P_HALF1, P_FULL0, P_FULL1, O_DONE, M_FULL0, M_FULL1, M_EMPTY0, M_EMPTY1, DRAIN, kNumBars };
+  static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag, [2] zero
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+__global__ void __launch_bounds__(kFwd256Threads, 1)
+    fwd_kernel_d256(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const FwdParams p) {
+  using S = Fwd256Smem;
+  constexpr int D = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_base_1024(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // grid (group * T_q, ceil(H / group), B); the query tiles of a head in longest-first order (the
+  // metadata orders pairs of tiles: pair = order[rank / 2], tile = 2 pair + rank % 2)
+  const int h = (int)blockIdx.y * p.group + (int)(blockIdx.x % p.group), b = blockIdx.z;
+  if (h >= p.H) return;
+  const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
+  const int rank = (int)(blockIdx.x / p.group);
+  const int qt = 2 * __ldg(p.order + bhm * p.n_pairs + rank / 2) + (rank & 1);
+  if (qt >= p.T_q) return;  // odd tile count: the pair's second tile does not exist
+  const int32_t* rows = p.row_entries + (bhm * p.T_q + qt) * p.T_k;
+  const int n = __ldg(p.row_count + bhm * p.T_q + qt);
+  const int ragged_kt = (p.n_k % kTile) ? p.T_k - 1 : -1;
+
+  const uint32_t bar0 = smem_u32(smem + S::kBar);
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + S::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  const volatile int* never = reinterpret_cast<const volatile int*>(misc + 2);
+  const uint32_t q_s = smem_u32(smem + S::kQ), k_s = smem_u32(smem + S::kK), v_s = smem_u32(smem + S::kV);
+  const int32_t* mask_smem = reinterpret_cast<const int32_t*>(smem + S::kMask);
+  uint16_t* list = reinterpret_cast<uint16_t*>(smem + S::kList);
+
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < S::kNumBars; ++k) mbar_init(bar(k), 1);
+    mbar_init(bar(S::P_HALF0), kTile);
+    mbar_init(bar(S::P_HALF1), kTile);
+    mbar_init(bar(S::P_FULL0), kTile);
+    mbar_init(bar(S::P_FULL1), kTile);
+    mbar_init(bar(S::M_EMPTY0), kTile);
+    mbar_init(bar(S::M_EMPTY1), kTile);
+    *abort_flag = 0;
+    misc[2] = 0;
+    fence_barrier_init();
+    if (n > 0) {
+      fence_proxy_async_smem();
+      prefetch_tmap(&tm_q);
+      mbar_arrive_expect_tx(bar(S::Q_FULL), 128 * D * 2);
+      for (int c = 0; c < 4; ++c) tma_load_4d(q_s + c * 16384, &tm_q, bar(S::Q_FULL), c * 64, h, qt * kTile, b);
+    }
+  }
+  for (int t = threadIdx.x; t < n; t += kFwd256Threads) list[t] = (uint16_t)__ldg(rows + t);
+  if (warp == 6) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int hk = h / p.q_per_kv;
+  // class of list entry e: 1 partial, 2 full (a ragged last key tile is always partial)
+  auto cls_of = [&](int e, int& kt) {
+    const int ent = list[e];
+    kt = ent >> 1;
+    return ((ent & 1) || kt == ragged_kt) ? 1 : 2;
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------- K and mask-slice loads (lane 0)
+    if (lane == 0 && n > 0) {
+      prefetch_tmap(&tm_k);
+      int nvec = 0;
+      for (int c = 0; c < 4; ++c) nvec += p.vec[c] ? 1 : 0;
+      bool ok = true;
+      int mcount = 0;
+      for (int e = 0; ok && e < n; ++e) {
+        int kt;
+        const int c = cls_of(e, kt);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int u = 2 * e + hh, slot = u & 1;
+          if (u >= 2 && !mbar_wait(bar(S::K_EMPTY0 + slot), ((u >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(S::K_FULL0 + slot), S::kHalfBytes);
+          for (int a = 0; a < 4; ++a)
+            tma_load_4d(k_s + slot * S::kHalfBytes + a * 8192, &tm_k, bar(S::K_FULL0 + slot), a * 64, hk,
+                        kt * kTile + hh * kHalf, b);
+        }
+        if (ok && c == 1) {
+          const int mb = mcount & 1;
+          if (mcount >= 2 && !mbar_wait(bar(S::M_EMPTY0 + mb), ((mcount >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t vbytes = 4u * (uint32_t)min(kTile, p.n_k - kt * kTile);
+          mbar_arrive_expect_tx(bar(S::M_FULL0 + mb), vbytes * nvec);
+          for (int v = 0; v < 4; ++v)
+            if (p.vec[v])
+              bulk_load(smem_u32(mask_smem + (mb * 4 + v) * kTile), p.vec[v] + bhm * p.n_k + (int64_t)kt * kTile,
+                        vbytes, bar(S::M_FULL0 + mb));
+          ++mcount;
+        }
+      }
+      if (!ok) record_failure(p.status, abort_flag, 21);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------- V loads (lane 0)
+    if (lane == 0 && n > 0) {
+      prefetch_tmap(&tm_v);
+      bool ok = true;
+      for (int e = 0; ok && e < n; ++e) {
+        int kt;
+        cls_of(e, kt);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int u = 2 * e + hh, slot = u & 1;
+          if (u >= 2 && !mbar_wait(bar(S::V_EMPTY0 + slot), ((u >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(S::V_FULL0 + slot), S::kHalfBytes);
+          for (int a = 0; a < 4; ++a)
+            tma_load_4d(v_s + slot * S::kHalfBytes + a * 8192, &tm_v, bar(S::V_FULL0 + slot), a * 64, hk,
+                        kt * kTile + hh * kHalf, b);
+        }
+      }
+      if (!ok) record_failure(p.status, abort_flag, 22);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ MMA role (lane 0)
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t kIdS = idesc_bf16(128, kHalf, false, false);  // S half: Q K-major, K K-major
+      constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);      // O += P V: V MN-major, N = 256
+      constexpr uint32_t kHi = desc_hi(1024);
+      const uint32_t lo_q = desc_lo(q_s, 16), lo_k = desc_lo(k_s, 16), lo_v = desc_lo(v_s, 8192);
+      constexpr uint32_t kHalfW = S::kHalfBytes >> 4;
+      auto issue_s = [&](int e) -> bool {  // S(e) into buffer e & 1: one N = 64 group per K half
+        const uint32_t tS = tmem + (e & 1) * 128;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int u = 2 * e + hh, slot = u & 1;
+          if (!mbar_wait(bar(S::K_FULL0 + slot), (u >> 1) & 1, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t oq = ((k >> 2) * 16384 + (k & 3) * 32) >> 4, ok_ = ((k >> 2) * 8192 + (k & 3) * 32) >> 4;
+            umma_ss_w<false>(tS + hh * kHalf, lo_q + oq, kHi, lo_k + slot * kHalfW + ok_, kHi, kIdS, k > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(S::K_EMPTY0 + slot));
+        }
+        umma_commit(bar(S::S_FULL0 + (e & 1)));
+        return true;
+      };
+      bool ok = mbar_wait(bar(S::Q_FULL), 0, abort_flag);
+      if (ok) ok = issue_s(0);
+      if (ok && n > 1) ok = issue_s(1);
+      for (int e = 0; ok && e < n; ++e) {
+        const int sb = e & 1, ph = (e >> 1) & 1;
+        const uint32_t tS = tmem + sb * 128, tO = tmem + 256;
+        // O += P(e) V(e): keys [0, 64) as soon as the first half of P is in TMEM, then keys [64, 128)
+        for (int hh = 0; ok && hh < 2; ++hh) {
+          const int u = 2 * e + hh, slot = u & 1;
+          if (!mbar_wait(bar(hh ? S::P_FULL0 + sb : S::P_HALF0 + sb), ph, abort_flag) ||
+              !mbar_wait(bar(S::V_FULL0 + slot), (u >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kHalf / 16; ++k)
+            umma_ts_w<false>(tO, tS + hh * 32 + k * 8, lo_v + slot * kHalfW + ((k * 16 * 128) >> 4), kHi, kIdPV,
+                             (e > 0 || hh > 0 || k > 0) ? 1u : 0u);
+          umma_commit(bar(S::V_EMPTY0 + slot));
+        }
+        if (!ok) break;
+        umma_commit(bar(S::O_DONE));
+        if (e + 2 < n) ok = issue_s(e + 2);  // after PV(e) has read P(e) from the same columns
+      }
+      if (!ok) record_failure(p.status, abort_flag, 23);
+      umma_commit(bar(S::DRAIN));
+      mbar_wait(bar(S::DRAIN), 0, never);
+    }
+  } else {
+    // ------------------------------------------------------ softmax role (warps 0-3)
+    const int r = threadIdx.x;  // row in tile == TMEM lane
+    const int i = qt * kTile + r;
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const uint32_t has = (p.vec[0] ? 1u : 0u) | (p.vec[1] ? 2u : 0u) | (p.vec[2] ? 4u : 0u) | (p.vec[3] ? 8u : 0u);
+    const uint32_t tO = tmem + 256 + lane_addr;
+    float m_run = kNegInf, l_run = 0.f, lq_run = 0.f;
+    int mcount = 0;
+    bool ok = true;
+    int e = 0;
+    for (; e < n; ++e) {
+      int kt;
+      const int ct = cls_of(e, kt);
+      const int sb = e & 1;
+      const uint32_t tS = tmem + sb * 128 + lane_addr;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(S::S_FULL0 + sb), (e >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld128(tS, s);
+      if (ct == 1) {
+        const int mb = mcount & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(S::M_FULL0 + mb), (mcount >> 1) & 1, abort_flag));
+        if (!ok) break;
+        const int32_t* mv = mask_smem + mb * 4 * kTile;
+        const int32_t w0 = qt * kTile + warp * 32;
+        uint32_t mw[4];
+#pragma unroll
+        for (int jb = 0; jb < 4; ++jb) {
+          const int c = jb * 32 + lane;
+          const int32_t lts = (has & 1u) ? mv[c] : p.n_q, lte = (has & 2u) ? mv[kTile + c] : p.n_q;
+          const int32_t uts = (has & 4u) ? mv[2 * kTile + c] : 0, ute = (has & 8u) ? mv[3 * kTile + c] : 0;
+          mw[jb] = interval_bits32(lts, lte, w0) | interval_bits32(uts, ute, w0);
+        }
+        bit_transpose32<4>(mw, lane);
+        if (kt == ragged_kt) {
+          const int valid = p.n_k - kt * kTile;
+#pragma unroll
+          for (int jb = 0; jb < 4; ++jb) {
+            const int v = valid - jb * 32;
+            mw[jb] |= v >= 32 ? 0u : (v <= 0 ? 0xFFFFFFFFu : ~((1u << v) - 1u));
+          }
+        }
+#pragma unroll
+        for (int jb = 0; jb < 4; ++jb) {
+          if (__any_sync(0xffffffffu, mw[jb] != 0u)) {
+#pragma unroll
+            for (int l = 0; l < 32; ++l) s[jb * 32 + l] = ((mw[jb] >> l) & 1u) ? __float_as_uint(kNegInf) : s[jb * 32 + l];
+          }
+        }
+        __syncwarp();
+        mbar_arrive(bar(S::M_EMPTY0 + mb));
+        ++mcount;
+      }
+      float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+      for (int c = 0; c < kTile; c += 8) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], __uint_as_float(s[c + 2 * u]), __uint_as_float(s[c + 2 * u + 1]));
+      }
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
+      const bool move = (m_tile - m_run) > kRescaleThreshold;
+      const float m_new = move ? m_tile : m_run;
+      const float alpha = move ? ex2(m_run - m_new) : 1.f;
+      const float m_use = (m_new == kNegInf) ? 0.f : m_new;
+      const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-m_use, -m_use);
+      uint64_t rs2[4] = {0, 0, 0, 0};
+      float rq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < kTile / 2; c += 2) {
+          const int cs = hh * (kTile / 2) + c;
+          const uint64_t x2 = fma2(((uint64_t)s[cs + 1] << 32) | s[cs], sc2, nm2);
+          float p0, p1;
+          if (((c >> 1) & (kPolyEvery - 1)) == kPolyEvery - 1) {
+            const uint64_t e2 = exp2_poly2(x2);
+            p0 = f2lo(e2);
+            p1 = f2hi(e2);
+          } else {
+            p0 = ex2(f2lo(x2));
+            p1 = ex2(f2hi(x2));
+          }
+          const int k = (c >> 1) & 3;
+          rs2[k] = add2(rs2[k], f2pack(p0, p1));
+          const uint32_t w = pack_bf16(p0, p1);
+          rq[k] = add_bf16x2_to_f32(w, rq[k]);
+          pk[c >> 1] = w;
+        }
+        if (hh == 0 && __any_sync(0xffffffffu, move && e > 0)) {
+          // O holds the sum over earlier tiles: wait for the last PV, rescale O in TMEM
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE), (e - 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t orr[32];
+            tmem_ld32(tO + cc * 32, orr);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) orr[c] = __float_as_uint(__uint_as_float(orr[c]) * alpha);
+            tmem_st32(tO + cc * 32, orr);
+          }
+        }
+        tmem_st32(tS + hh * 32, pk);
+        tc_fence_before();
+        mbar_arrive(bar((hh ? S::P_FULL0 : S::P_HALF0) + sb));
+      }
+      if (!ok) break;
+      const uint64_t rs2a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
+      l_run = l_run * alpha + (f2lo(rs2a) + f2hi(rs2a));
+      lq_run = lq_run * alpha + ((rq[0] + rq[1]) + (rq[2] + rq[3]));
+      m_run = m_new;
+    }
+    if (!ok) record_failure(p.status, abort_flag, 24);
+    // epilogue: O = O / l staged in the Q buffer (every S product has finished once the last PV
+    // has), TMA-stored by one thread; LSE = (m + log2 l) ln 2; empty rows: O = 0, LSE = -inf
+    const bool live = ok && n > 0 && l_run > kLiveSum;
+    bool have_o = false;
+    if (ok && n > 0) {
+      have_o = __all_sync(0xffffffffu, mbar_wait(bar(S::O_DONE), (n - 1) & 1, abort_flag));
+      if (!have_o) record_failure(p.status, abort_flag, 25);
+      tc_fence_after();
+    }
+    const float inv = live ? 1.f / lq_run : 0.f;
+    uint8_t* stage = smem + S::kQ;
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t orr[32];
+      if (have_o) {
+        tmem_ld32(tO + cc * 32, orr);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) orr[c] = 0u;
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) pk[c >> 1] = pack_bf16(__uint_as_float(orr[c]) * inv, __uint_as_float(orr[c + 1]) * inv);
+      uint8_t* row = stage + (cc >> 1) * 16384 + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch)
+        *reinterpret_cast<uint4*>(row + ((((cc & 1) * 4 + ch) ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(2, 128);
+    if (r == 0) {
+      for (int c = 0; c < 4; ++c) tma_store_4d(&tm_o, smem_u32(stage + c * 16384), c * 64, h, qt * kTile, b);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+    if (i < p.n_q)
+      p.lse[((int64_t)b * p.H + h) * p.n_q + (int64_t)i] = live ? (m_run + __log2f(l_run)) * 0.69314718055994531f : kNegInf;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 6) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+fm_status launch_fwd_d256(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], void* o,
+                          float* lse, cudaStream_t stream) {
+  using S = Fwd256Smem;
+  static_assert(S::kAlloc <= 227 * 1024, "forward (D = 256) shared memory exceeds the per-CTA limit");
+  constexpr int D = 256;
+  CUtensorMap tq, tk, tv, to;
+  const int H_kv = a->H_kv ? a->H_kv : a->H;
+  if (!encode_tmap_bf16_4d(&tq, a->q, D, a->H, a->n_q, a->B, kTile) ||
+      !encode_tmap_bf16_4d(&tk, a->k, D, H_kv, a->n_k, a->B, kHalf) ||
+      !encode_tmap_bf16_4d(&tv, a->v, D, H_kv, a->n_k, a->B, kHalf) ||
+      !encode_tmap_bf16_4d(&to, o, D, a->H, a->n_q, a->B, kTile))
+    return FM_ERR_CUDA;
+  FwdParams p;
+  p.row_count = meta->row_count;
+  p.row_entries = meta->row_entries;
+  p.order = meta->fwd_order;
+  for (int c = 0; c < 4; ++c) p.vec[c] = vec ? vec[c] : nullptr;
+  p.v32 = nullptr;
+  p.o = o;
+  p.lse = lse;
+  p.status = device_status_ptr();
+  p.B = a->B;
+  p.H = a->H;
+  p.H_kv = H_kv;
+  p.q_per_kv = a->H / H_kv;
+  p.Hm = meta->d.Hm;
+  p.n_q = a->n_q;
+  p.n_k = a->n_k;
+  p.T_q = (a->n_q + kTile - 1) / kTile;
+  p.T_k = (a->n_k + kTile - 1) / kTile;
+  p.n_pairs = (p.T_q + 1) / 2;
+  p.group = dispatch_group(p.H, 2.0 * a->n_k * D * 2);
+  p.scale_log2 = a->scale * 1.4426950408889634f;
+  if (!smem_opt_in<fwd_kernel_d256>(S::kAlloc)) return FM_ERR_CUDA;
+  const int ranks = 2 * p.n_pairs;  // query tiles rounded up to whole pairs
+  fwd_kernel_d256<<<dim3(p.group * ranks, (p.H + p.group - 1) / p.group, p.B), kFwd256Threads, S::kAlloc, stream>>>(
+      tq, tk, tv, to, p);
+  return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
+}
+
 template <int D, bool F32>
 fm_status launch_fwd(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4], void* o,
                      float* lse, cudaStream_t stream) {
@@ -620,8 +1031,8 @@ fm_status check_attn_args(const fm_attn_args* a, const fm_mask_meta* meta, const
   if (a->B < 1 || a->H < 1 || a->n_q < 1 || a->n_k < 1 || a->B > 65535 || a->H > 65535) return FM_ERR_INVALID_ARG;
   if (!(a->scale > 0.f) || a->scale > 3.0e38f) return FM_ERR_INVALID_ARG;  // positive and finite
   if (a->dtype != 0 && a->dtype != 1) return FM_ERR_UNSUPPORTED;
-  if (a->D != 64 && a->D != 128) return FM_ERR_UNSUPPORTED;
-  if (a->dtype == 1 && a->D != 64) return FM_ERR_UNSUPPORTED;  // fp32 tiles of D=128 exceed shared memory
+  if (a->D != 64 && a->D != 128 && a->D != 256) return FM_ERR_UNSUPPORTED;
+  if (a->dtype == 1 && a->D != 64) return FM_ERR_UNSUPPORTED;  // fp32 tiles of D >= 128 exceed shared memory
   if (a->n_k % 4) return FM_ERR_UNSUPPORTED;  // key tiles' bound vectors are staged by 16-byte bulk copies
   if ((a->n_k + kTile - 1) / kTile > kMaxList || (a->n_q + kTile - 1) / kTile > kMaxList)
     return FM_ERR_UNSUPPORTED;  // lists held in smem
@@ -655,6 +1066,7 @@ extern "C" fm_status fm_attn_fwd(const fm_attn_args* a, const fm_mask_meta* meta
     return FM_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (a->dtype == 1) return fm::launch_fwd<64, true>(a, meta, vec, o, lse, s);
+  if (a->D == 256) return fm::launch_fwd_d256(a, meta, vec, o, lse, s);
   return a->D == 64 ? fm::launch_fwd<64, false>(a, meta, vec, o, lse, s)
                     : fm::launch_fwd<128, false>(a, meta, vec, o, lse, s);
 }

@@ -17,6 +17,7 @@ constexpr int kTile = 128;
 
 struct MetaParams {
   const int32_t* vec[4];  // [B, Hm, n_k] or null
+  bool vec16;             // every vector row starts 16-byte aligned (n_k % 4 == 0): 16-byte loads
   int32_t* minmax;        // [BHm, T_k, 8]
   uint8_t* cls;           // [BHm, T_q, T_k]
   int32_t* row_count;     // [BHm, T_q]
@@ -25,6 +26,7 @@ struct MetaParams {
   int32_t* col_entries;   // [BHm, T_k, T_q]
   int32_t* fwd_order;     // [BHm, ceil(T_q / 2)]
   int32_t* bwd_order;     // [BHm, T_k]
+  int32_t* done;          // [BHm] query-tile CTAs finished (the last one sorts the dispatch orders)
   int32_t BHm, n_q, n_k, T_q, T_k;
 };
 
@@ -32,12 +34,26 @@ __device__ __forceinline__ int32_t vec_at(const int32_t* v, int64_t idx, int32_t
   return v ? __ldg(v + idx) : dflt;
 }
 
-// One warp per key tile: lanes stride over the tile's 128 columns.
-__global__ void __launch_bounds__(256) meta_minmax_kernel(const MetaParams p) {
+// 0 skip, 1 partial, 2 full for query rows [r0, r1) against one key tile's min/max.
+__device__ __forceinline__ int classify(const int4 lo, const int4 hi, int64_t r0, int64_t r1) {
+  // lo = (minLTS, maxLTS, minLTE, maxLTE), hi = (minUTS, maxUTS, minUTE, maxUTE)
+  const bool skip = ((int64_t)lo.y <= r0 && (int64_t)lo.z >= r1) || ((int64_t)hi.y <= r0 && (int64_t)hi.z >= r1);
+  const bool clear_l = ((int64_t)lo.x >= r1) || ((int64_t)lo.w <= r0);
+  const bool clear_u = ((int64_t)hi.x >= r1) || ((int64_t)hi.w <= r0);
+  return skip ? 0 : ((clear_l && clear_u) ? 2 : 1);
+}
+
+// Key-tile pass: one warp per (bhm, key tile).  Min and max of the four vectors over the tile's 128
+// columns (one 16-byte load per lane and vector when the rows are 16-byte aligned), written to
+// minmax, then the tile's column list: every query tile classified against those eight values,
+// 32 per step, the non-skip ones compacted in ascending order.  Also clears the per-bhm counter
+// of the query-tile pass.
+__global__ void __launch_bounds__(256) meta_cols_kernel(const MetaParams p) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= p.BHm * p.T_k) return;
   const int bhm = warp / p.T_k, kt = warp % p.T_k;
+  if (kt == 0 && lane == 0) p.done[bhm] = 0;
   const int32_t dflt[4] = {p.n_q, p.n_q, 0, 0};
   int32_t mn[4], mx[4];
 #pragma unroll
@@ -46,14 +62,28 @@ __global__ void __launch_bounds__(256) meta_minmax_kernel(const MetaParams p) {
     mx[c] = INT_MIN;
   }
   const int64_t base = (int64_t)bhm * p.n_k;
-  for (int t = lane; t < kTile; t += 32) {
-    const int64_t j = (int64_t)kt * kTile + t;
-    if (j >= p.n_k) break;
+  const int64_t j0 = (int64_t)kt * kTile;
+  if (p.vec16) {
+    const int64_t j = j0 + 4 * lane;  // n_k % 4 == 0: a group of 4 is either inside or past the end
+    if (j < p.n_k) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int32_t v = vec_at(p.vec[c], base + j, dflt[c]);
-      mn[c] = min(mn[c], v);
-      mx[c] = max(mx[c], v);
+      for (int c = 0; c < 4; ++c) {
+        int4 v = make_int4(dflt[c], dflt[c], dflt[c], dflt[c]);
+        if (p.vec[c]) v = __ldg(reinterpret_cast<const int4*>(p.vec[c] + base + j));
+        mn[c] = min(min(v.x, v.y), min(v.z, v.w));
+        mx[c] = max(max(v.x, v.y), max(v.z, v.w));
+      }
+    }
+  } else {
+    for (int t = lane; t < kTile; t += 32) {
+      const int64_t j = j0 + t;
+      if (j >= p.n_k) break;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int32_t v = vec_at(p.vec[c], base + j, dflt[c]);
+        mn[c] = min(mn[c], v);
+        mx[c] = max(mx[c], v);
+      }
     }
   }
 #pragma unroll
@@ -73,26 +103,79 @@ __global__ void __launch_bounds__(256) meta_minmax_kernel(const MetaParams p) {
     val = (c == 3) ? ((lane & 1) ? mx[3] : mn[3]) : val;
     p.minmax[((int64_t)bhm * p.T_k + kt) * 8 + lane] = val;
   }
-}
-
-// 0 skip, 1 partial, 2 full for query rows [r0, r1) against one key tile's min/max.
-__device__ __forceinline__ int classify(const int4 lo, const int4 hi, int64_t r0, int64_t r1) {
-  // lo = (minLTS, maxLTS, minLTE, maxLTE), hi = (minUTS, maxUTS, minUTE, maxUTE)
-  const bool skip = ((int64_t)lo.y <= r0 && (int64_t)lo.z >= r1) || ((int64_t)hi.y <= r0 && (int64_t)hi.z >= r1);
-  const bool clear_l = ((int64_t)lo.x >= r1) || ((int64_t)lo.w <= r0);
-  const bool clear_u = ((int64_t)hi.x >= r1) || ((int64_t)hi.w <= r0);
-  return skip ? 0 : ((clear_l && clear_u) ? 2 : 1);
-}
-
-// Row lists (blockIdx.y == 0): one warp per (bhm, query tile), scanning key
-// tiles 32 at a time; column lists (blockIdx.y == 1): one warp per (bhm, key tile).
-__global__ void __launch_bounds__(256) meta_lists_kernel(const MetaParams p) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+  // column list of this key tile
+  const int4 lo = make_int4(mn[0], mx[0], mn[1], mx[1]), hi = make_int4(mn[2], mx[2], mn[3], mx[3]);
   const unsigned below = (1u << lane) - 1u;
-  if (blockIdx.y == 0) {
-    if (warp >= p.BHm * p.T_q) return;
-    const int bhm = warp / p.T_q, qt = warp % p.T_q;
+  int32_t* ent = p.col_entries + ((int64_t)bhm * p.T_k + kt) * p.T_q;
+  int count = 0;
+  for (int q0 = 0; q0 < p.T_q; q0 += 32) {
+    const int qt = q0 + lane;
+    int c = 0;
+    if (qt < p.T_q) {
+      const int64_t r0 = (int64_t)qt * kTile, r1 = (r0 + kTile < p.n_q) ? r0 + kTile : (int64_t)p.n_q;
+      c = classify(lo, hi, r0, r1);
+    }
+    const unsigned keep = __ballot_sync(0xffffffffu, c != 0);
+    if (c != 0) ent[count + __popc(keep & below)] = (qt << 1) | (c == 1 ? 1 : 0);
+    count += __popc(keep);
+  }
+  if (lane == 0) p.col_count[(int64_t)bhm * p.T_k + kt] = count;
+}
+
+// Dispatch orders (longest first) of one (b, hm), by the CTA that finishes the query-tile pass
+// last: the forward's query-tile pairs by the sum of their two row counts, the backward's key
+// tiles by column count; ties keep ascending index.  Bitonic sort in shared memory of the keys
+// (cost << 16) | (0xFFFF - index), descending; with at most 4096 items and costs below 2^16 the
+// keys are distinct, so the order is deterministic.  The two sorts run side by side, each on 512
+// threads of the CTA and its own named barrier.
+constexpr int kOrderMax = 4096;
+constexpr int kRowsThreads = 1024;
+__device__ void sort_order(uint32_t* key, const int32_t* cost_a, bool pairs, int n, int n_b, int32_t* out, int tid,
+                           int bar_id) {
+  constexpr int kT = kRowsThreads / 2;
+  int np2 = 1;
+  while (np2 < n) np2 <<= 1;
+  for (int i = tid; i < np2; i += kT) {
+    uint32_t k = 0;  // padding sorts last
+    if (i < n) {
+      // counts written by other CTAs of this launch: read through L2 (__ldcg), not a stale L1 line
+      const uint32_t cost = pairs ? (uint32_t)(__ldcg(cost_a + 2 * i) + (2 * i + 1 < n_b ? __ldcg(cost_a + 2 * i + 1) : 0))
+                                  : (uint32_t)__ldcg(cost_a + i);
+      k = (cost << 16) | (0xFFFFu - (uint32_t)i);
+    }
+    key[i] = k;
+  }
+  named_bar_sync(bar_id, kT);
+  for (int len = 2; len <= np2; len <<= 1) {
+    for (int j = len >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < np2; i += kT) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint32_t a = key[i], b = key[ixj];
+          const bool desc = (i & len) == 0;  // descending runs merge into one descending sequence
+          if (desc ? (a < b) : (a > b)) {
+            key[i] = b;
+            key[ixj] = a;
+          }
+        }
+      }
+      named_bar_sync(bar_id, kT);
+    }
+  }
+  for (int i = tid; i < n; i += kT) out[i] = (int32_t)(0xFFFFu - (key[i] & 0xFFFFu));
+}
+
+// Query-tile pass: grid (ceil(T_q / 32), BHm), 1024 threads, one warp per query tile: its row of the
+// class matrix and its row list (key tiles scanned 32 at a time against the key-tile pass's min/max).
+// The CTA that completes a (b, hm) last also writes that (b, hm)'s two dispatch orders.
+__global__ void __launch_bounds__(kRowsThreads) meta_rows_kernel(const MetaParams p) {
+  __shared__ uint32_t key_f[kOrderMax / 2];
+  __shared__ uint32_t key_b[kOrderMax];
+  __shared__ int last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bhm = blockIdx.y, qt = blockIdx.x * (kRowsThreads / 32) + warp;
+  const unsigned below = (1u << lane) - 1u;
+  if (qt < p.T_q) {
     const int64_t r0 = (int64_t)qt * kTile, r1 = (r0 + kTile < p.n_q) ? r0 + kTile : (int64_t)p.n_q;
     const int4* mm = reinterpret_cast<const int4*>(p.minmax + (int64_t)bhm * p.T_k * 8);
     uint8_t* cls = p.cls + ((int64_t)bhm * p.T_q + qt) * p.T_k;
@@ -110,26 +193,28 @@ __global__ void __launch_bounds__(256) meta_lists_kernel(const MetaParams p) {
       count += __popc(keep);
     }
     if (lane == 0) p.row_count[(int64_t)bhm * p.T_q + qt] = count;
-  } else {
-    if (warp >= p.BHm * p.T_k) return;
-    const int bhm = warp / p.T_k, kt = warp % p.T_k;
-    const int4* mm = reinterpret_cast<const int4*>(p.minmax + ((int64_t)bhm * p.T_k + kt) * 8);
-    const int4 lo = __ldg(mm), hi = __ldg(mm + 1);
-    int32_t* ent = p.col_entries + ((int64_t)bhm * p.T_k + kt) * p.T_q;
-    int count = 0;
-    for (int q0 = 0; q0 < p.T_q; q0 += 32) {
-      const int qt = q0 + lane;
-      int c = 0;
-      if (qt < p.T_q) {
-        const int64_t r0 = (int64_t)qt * kTile, r1 = (r0 + kTile < p.n_q) ? r0 + kTile : (int64_t)p.n_q;
-        c = classify(lo, hi, r0, r1);
-      }
-      const unsigned keep = __ballot_sync(0xffffffffu, c != 0);
-      if (c != 0) ent[count + __popc(keep & below)] = (qt << 1) | (c == 1 ? 1 : 0);
-      count += __popc(keep);
-    }
-    if (lane == 0) p.col_count[(int64_t)bhm * p.T_k + kt] = count;
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's counts before its arrival
+    last = atomicAdd(p.done + bhm, 1) == (int)gridDim.x - 1;
+    if (last) __threadfence();  // every other CTA's counts after it
+  }
+  __syncthreads();
+  if (!last) return;
+  const int n_pairs = (p.T_q + 1) / 2;
+  int32_t* fo = p.fwd_order + (int64_t)bhm * n_pairs;
+  int32_t* bo = p.bwd_order + (int64_t)bhm * p.T_k;
+  if (p.T_q > kOrderMax || p.T_k > kOrderMax) {  // sizes the attention kernels do not take
+    for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) fo[i] = i;
+    for (int i = threadIdx.x; i < p.T_k; i += blockDim.x) bo[i] = i;
+    return;
+  }
+  constexpr int kT = kRowsThreads / 2;
+  if (threadIdx.x < kT)
+    sort_order(key_f, p.row_count + (int64_t)bhm * p.T_q, true, n_pairs, p.T_q, fo, threadIdx.x, 1);
+  else
+    sort_order(key_b, p.col_count + (int64_t)bhm * p.T_k, false, p.T_k, 0, bo, threadIdx.x - kT, 2);
 }
 
 // Packed variable-length batch -> document-mask vectors, one thread per key: the key's sequence is
@@ -160,57 +245,8 @@ __global__ void __launch_bounds__(256) varlen_mask_kernel(const int32_t* __restr
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Dispatch orders for the attention kernels (longest first).  One CTA per
-// (b, hm) and direction: blockIdx.y = 0 orders query-tile pairs by the sum of
-// their two row counts, 1 orders key tiles by column count; ties keep
-// ascending index.  Bitonic sort in shared memory of the keys
-// (cost << 16) | (0xFFFF - index), descending; with at most 4096 items and
-// costs below 2^16 the keys are distinct, so the order is deterministic.
-constexpr int kOrderMax = 4096;
-__global__ void __launch_bounds__(1024) meta_order_kernel(const MetaParams p) {
-  __shared__ uint32_t key[kOrderMax];
-  const int bhm = blockIdx.x;
-  const bool fwd = blockIdx.y == 0;
-  const int n = fwd ? (p.T_q + 1) / 2 : p.T_k;
-  int32_t* out = fwd ? p.fwd_order + (int64_t)bhm * n : p.bwd_order + (int64_t)bhm * n;
-  if (p.T_q > kOrderMax || p.T_k > kOrderMax) {  // sizes the attention kernels do not take
-    for (int i = threadIdx.x; i < n; i += blockDim.x) out[i] = i;
-    return;
-  }
-  int np2 = 1;
-  while (np2 < n) np2 <<= 1;
-  const int32_t* rc = p.row_count + (int64_t)bhm * p.T_q;
-  const int32_t* cc = p.col_count + (int64_t)bhm * p.T_k;
-  for (int i = threadIdx.x; i < np2; i += blockDim.x) {
-    uint32_t k = 0;  // padding sorts last
-    if (i < n) {
-      const uint32_t cost = fwd ? (uint32_t)(rc[2 * i] + (2 * i + 1 < p.T_q ? rc[2 * i + 1] : 0)) : (uint32_t)cc[i];
-      k = (cost << 16) | (0xFFFFu - (uint32_t)i);
-    }
-    key[i] = k;
-  }
-  __syncthreads();
-  for (int len = 2; len <= np2; len <<= 1) {
-    for (int j = len >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < np2; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint32_t a = key[i], b = key[ixj];
-          const bool desc = (i & len) == 0;  // descending runs merge into one descending sequence
-          if (desc ? (a < b) : (a > b)) {
-            key[i] = b;
-            key[ixj] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  for (int i = threadIdx.x; i < n; i += blockDim.x) out[i] = (int32_t)(0xFFFFu - (key[i] & 0xFFFFu));
-}
-
 struct MetaLayout {
-  size_t minmax, row_count, row_entries, col_count, col_entries, cls, fwd_order, bwd_order, total;
+  size_t minmax, row_count, row_entries, col_count, col_entries, cls, fwd_order, bwd_order, done, total;
 };
 
 bool meta_layout(const fm_mask_desc* d, MetaLayout* L) {
@@ -236,6 +272,8 @@ bool meta_layout(const fm_mask_desc* d, MetaLayout* L) {
   off = align256(off + BHm * ((T_q + 1) / 2) * 4);
   L->bwd_order = off;
   off = align256(off + BHm * T_k * 4);
+  L->done = off;
+  off = align256(off + BHm * 4);
   L->total = off;
   return true;
 }
@@ -280,17 +318,20 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
   p.col_entries = out->col_entries;
   p.fwd_order = out->fwd_order;
   p.bwd_order = out->bwd_order;
+  p.done = reinterpret_cast<int32_t*>(w + L.done);
   p.BHm = d->B * d->Hm;
   p.n_q = d->n_q;
   p.n_k = d->n_k;
   p.T_q = (d->n_q + fm::kTile - 1) / fm::kTile;
   p.T_k = (d->n_k + fm::kTile - 1) / fm::kTile;
+  uintptr_t al = (uintptr_t)(d->n_k % 4);
+  for (int c = 0; c < 4; ++c) al |= reinterpret_cast<uintptr_t>(p.vec[c]) & 15u;
+  p.vec16 = al == 0;
+  if (p.BHm > 65535) return FM_ERR_UNSUPPORTED;  // grid.y of the query-tile pass
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t warps_mm = (int64_t)p.BHm * p.T_k;
-  fm::meta_minmax_kernel<<<(unsigned)((warps_mm + 7) / 8), 256, 0, s>>>(p);
-  const int64_t warps_l = (int64_t)p.BHm * (p.T_q > p.T_k ? p.T_q : p.T_k);
-  fm::meta_lists_kernel<<<dim3((unsigned)((warps_l + 7) / 8), 2), 256, 0, s>>>(p);
-  fm::meta_order_kernel<<<dim3((unsigned)p.BHm, 2), 1024, 0, s>>>(p);
+  const int64_t warps_k = (int64_t)p.BHm * p.T_k;
+  fm::meta_cols_kernel<<<(unsigned)((warps_k + 7) / 8), 256, 0, s>>>(p);
+  fm::meta_rows_kernel<<<dim3((unsigned)((p.T_q + 31) / 32), (unsigned)p.BHm), fm::kRowsThreads, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

@@ -255,6 +255,16 @@ def test_tiny_causal_document(fm, D):
     _compare(res, vecs, 1)
 
 
+@pytest.mark.parametrize("n,family", [(256, "causal_document"), (640, "full"), (640, "sliding_window_2k"),
+                                      (1000, "random_eviction"), (388, "share_question"), (1536, "global_sliding")])
+def test_head_dim_256_forward(fm, n, family):
+    """D = 256 (one query tile per CTA, K / V streamed in 64-key halves): the forward against the
+    oracle on every row of both heads, ragged lengths included."""
+    vecs = _vec_stack(synth.make_family(family, n, 71), 1, 1)
+    res = _run_attention(fm, 1, 2, n, n, 256, vecs, 1, seed=72, bwd=False)
+    _compare(res, vecs, 1, bwd=False)
+
+
 def _run_fp32(fm, B, H, n, vecs, seed):
     """fp32 inputs and outputs (tf32 tensor-core products), D = 64."""
     D = 64

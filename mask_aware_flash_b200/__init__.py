@@ -28,7 +28,7 @@ _lib = None
 FM_OK, FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA, FM_ERR_DEVICE_TIMEOUT = range(6)
 TILE = 128
 META_LAUNCHES = 2  # kernels one fm_build_mask_meta call launches
-BWD_LAUNCHES = 2   # kernels one fm_attn_bwd call launches (one more with deterministic=True)
+BWD_LAUNCHES = 3   # kernels one fm_attn_bwd call launches (one more with deterministic=True)
 
 
 class FmError(RuntimeError):

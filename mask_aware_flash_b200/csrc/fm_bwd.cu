@@ -20,12 +20,8 @@
 // Warps 0-3 / 4-7 each take 32 of the 64 queries of a sub-tile; warp 12 issues
 // the TMA loads, warp 13 the MMAs.  A preprocess kernel forms D_i = dO_i.O_i
 // and the log2-domain LSE (rows padded to whole query tiles) and clears the
-// per-query-tile counters.  The first key tile to reach a query tile stores its
-// dQ contribution into the accumulator instead of adding it (so the
-// accumulator needs no clearing pass), and the last one, found by a counter of
-// completed contributors, scales that tile into dQ while it is still in L2 (so
-// no separate convert pass re-reads it).  The fp32 path (kind::tf32)
-// transposes its MN-major operands in shared memory (drain warps).
+// accumulator; a final kernel scales the accumulator into dQ.  The fp32 path
+// (kind::tf32) transposes its MN-major operands in shared memory (drain warps).
 #include "fm_common.cuh"
 
 namespace fm {
@@ -46,10 +42,7 @@ struct BwdParams {
   const int32_t* order;        // [B, Hm, T_k] dispatch order (longest first); null = ascending
   const uint16_t* turn;        // fixed-order dQ: [B, Hm, T_k, T_q] position of key tile kt in the
                                // row list of query tile qt; null = unordered adds
-  const int32_t* row_count;    // [B, Hm, T_q] key tiles contributing to each query tile
-  int* dq_ticket;              // [B, H, T_q] arrival tickets (unordered adds): ticket 0 stores
-  int* dq_done;                // [B, H, T_q] contributors whose dQ adds are complete (fixed order: the turn)
-  void* dq;                    // [B, n_q, H, D] output, bf16 or fp32
+  int* dq_sem;                 // fixed-order dQ: [B, H, T_q] key tiles added so far per query tile
   const int32_t* vec[4];       // [B, Hm, n_k] or null
   const float* lse2;           // [B, H, n_q] log2-domain LSE, +inf on empty rows
   const float* dvec;           // [B, H, n_q] D_i = dO_i . O_i
@@ -89,9 +82,8 @@ struct BwdSmem {
          DS_READY, DS_EMPTY0, DS_EMPTY1, DQ_FULL, DQ_EMPTY, ACC_FULL, DRAIN,
          QT_GO0, QT_GO1, QT_READY0, QT_READY1, KT_READY,  // fp32 path: operand transposes
          kNumBars };
-  // [0] TMEM base, [1] abort, [2] zero flag, [3] / [4] drain broadcast slots (first / last contributor)
-  static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kBytes = kMisc + 32;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort, [2] zero flag
+  static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -132,41 +124,6 @@ __device__ __forceinline__ void transpose_k_f32(const uint8_t* k, uint8_t* kt, i
     const int e = it * 128 + tid, key = e >> 6, d = e & 63;
     const float x = *reinterpret_cast<const float*>(k + f32_sw128_off(key, d, kTile));
     *reinterpret_cast<uint32_t*>(kt + f32_sw128_off(d, key, 64)) = round_tf32(x);
-  }
-}
-
-// dQ rows [r0, r0 + 128) of head bh from the fp32 accumulator (two 64-row blocks, each
-// [16 groups of 4 rows][D][4]): dQ = scale * acc, rows past n_q dropped.  128 threads; a work item
-// is (group g, 8 consecutive d): eight 16-byte L2 reads (4 rows x 8 d) and four 8-element row
-// stores.  The accumulator is read through L2 only (other SMs wrote it).
-template <int D, bool F32>
-__device__ __forceinline__ void convert_dq_tile(const float* acc_bh, void* dq, int b, int hq, int H, int n_q, int r0,
-                                                float scale, int tid) {
-  constexpr int kChunks = D / 8;
-#pragma unroll 1
-  for (int w = tid; w < 2 * 16 * kChunks; w += 128) {
-    const int blk = w / (16 * kChunks), g = (w / kChunks) % 16, c = w % kChunks;
-    const float4* src = reinterpret_cast<const float4*>(acc_bh + (int64_t)(r0 + 64 * blk) * D) + g * D + c * 8;
-    float4 x[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + u);
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int row = r0 + 64 * blk + 4 * g + r;
-      if (row >= n_q) continue;
-      float y[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) y[u] = (r == 0 ? x[u].x : r == 1 ? x[u].y : r == 2 ? x[u].z : x[u].w) * scale;
-      const int64_t off = (((int64_t)b * n_q + row) * H + hq) * D + c * 8;
-      if constexpr (F32) {
-        float* o = static_cast<float*>(dq) + off;
-        st_global_v4(o, __float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]), __float_as_uint(y[3]));
-        st_global_v4(o + 4, __float_as_uint(y[4]), __float_as_uint(y[5]), __float_as_uint(y[6]), __float_as_uint(y[7]));
-      } else {
-        st_global_v4(static_cast<__nv_bfloat16*>(dq) + off, pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]),
-                     pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]));
-      }
-    }
   }
 }
 
@@ -558,16 +515,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-    // Per query tile (two sub-tiles): the first contributor stores, later ones add once the first
-    // one's stores are complete; the contributor that completes the tile converts it into dQ.
-    volatile int* slot_first = reinterpret_cast<volatile int*>(misc + 3);
-    volatile int* slot_last = reinterpret_cast<volatile int*>(misc + 4);
-    bool first = false;
     for (int i = 0; ok && i < nsub; ++i) {
-      const int q0 = sub_q0(i), qt = q0 >> 7;
-      const int hq = hq0 + (G > 1 ? head_of(i, jh) : 0);
-      const int64_t bh = (int64_t)b * p.H + hq;
-      const int64_t ci = bh * p.T_q + qt;  // this query tile's counters
+      const int q0 = sub_q0(i);
+      const int64_t bh = (int64_t)b * p.H + hq0 + (G > 1 ? head_of(i, jh) : 0);
       float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q_pad * D;
       if constexpr (F32) {
         const int st = i % NS;
@@ -578,57 +528,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(bar(S::QT_READY0 + st));
       }
-      // a vote of all 128 drain threads (not per warp): they meet at named barriers below, so they
-      // must leave the loop together
-      ok = all_drain_threads(mbar_wait(bar(S::DQ_FULL), i & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(S::DQ_FULL), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t a[64];
       tmem_ld64(tdQ + lane_addr, a);
       tc_fence_before();
       mbar_arrive(bar(S::DQ_EMPTY));
-      if ((i & 1) == 0) {
-        if (p.turn) {  // fixed order: wait until the key tiles before this one have added
-          ok = all_drain_threads(d != 0 || flag_wait_eq(p.dq_done + ci, turn[i >> 1], p.status, abort_flag));
-          first = turn[i >> 1] == 0;
-        } else {
-          if (d == 0) *slot_first = atomicAdd(p.dq_ticket + ci, 1);
-          all_drain_threads(true);
-          first = *slot_first == 0;
-          ok = all_drain_threads(d != 0 || first || flag_wait_ge(p.dq_done + ci, 1, p.status, abort_flag));
-        }
+      int* sem = p.dq_sem ? p.dq_sem + bh * p.T_q + (q0 >> 7) : nullptr;
+      if (sem && (i & 1) == 0) {  // fixed order: wait until the key tiles before this one have added
+        ok = all_drain_threads(d != 0 || flag_wait_eq(sem, turn[i >> 1], p.status, abort_flag));
         if (!ok) break;
       }
       if (d < D) {
         float* blk = acc_bh + (int64_t)q0 * D;  // [16 groups of 4 queries][D][4]
-        if (first) {
 #pragma unroll
-          for (int g = 0; g < 16; ++g)
-            st_global_v4(blk + (g * D + d) * 4, a[4 * g], a[4 * g + 1], a[4 * g + 2], a[4 * g + 3]);
-        } else {
-#pragma unroll
-          for (int g = 0; g < 16; ++g)
-            red_add_v4(blk + (g * D + d) * 4, __uint_as_float(a[4 * g]), __uint_as_float(a[4 * g + 1]),
-                       __uint_as_float(a[4 * g + 2]), __uint_as_float(a[4 * g + 3]));
-        }
+        for (int g = 0; g < 16; ++g)
+          red_add_v4(blk + (g * D + d) * 4, __uint_as_float(a[4 * g]), __uint_as_float(a[4 * g + 1]),
+                     __uint_as_float(a[4 * g + 2]), __uint_as_float(a[4 * g + 3]));
       }
-      if ((i & 1) == 1) {  // both sub-tiles written: count this contributor; the last one converts
+      if (sem && (i & 1) == 1) {  // both sub-tiles added: pass the query tile on to the next key tile
         all_drain_threads(true);
-        if (d == 0) {
-          const int need = __ldg(p.row_count + bhm_of(hq) * p.T_q + qt);
-          __threadfence();
-          int done;
-          if (p.turn) {
-            done = turn[i >> 1] + 1;
-            st_release_gpu(p.dq_done + ci, done);
-          } else {
-            done = atomicAdd(p.dq_done + ci, 1) + 1;
-          }
-          *slot_last = done == need;
-          if (done == need) __threadfence();
-        }
-        all_drain_threads(true);
-        if (*slot_last) convert_dq_tile<D, F32>(acc_bh, p.dq, b, hq, p.H, p.n_q, qt * kTile, p.scale, d);
+        if (d == 0) st_release_gpu(sem, turn[i >> 1] + 1);
       }
     }
     if (!ok) record_failure(p.status, abort_flag, 14);
@@ -698,41 +619,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-// D_i = dO_i . O_i, log2-domain LSE (+inf for empty rows so that P = 0), cleared per-query-tile
-// counters, and dQ = 0 on the rows of query tiles that no key tile reaches (skip tiles only: no
-// contributor would write them).  One thread per (b, i, h) row.
-struct PrepParams {
-  const void* o;
-  const void* dout;
-  const float* lse;
-  float* lse2;
-  float* dvec;
-  int* counters;              // 2 x [B, H, T_q] (tickets, done)
-  const int32_t* row_count;   // [B, Hm, T_q]
-  void* dq;                   // [B, n_q, H, D]
-  int B, H, Hm, n_q, n_q_pad, T_q;
-};
-
+// D_i = dO_i . O_i, log2-domain LSE (+inf for empty rows so that P = 0), and
+// a cleared dQ accumulator.  One thread per (b, i, h) row.
 template <int D, bool F32>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepParams p) {
-  const int64_t rows = (int64_t)p.B * p.n_q * p.H;
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ o, const void* __restrict__ dout,
+                                                       const float* __restrict__ lse, float* __restrict__ lse2,
+                                                       float* __restrict__ dvec, float* __restrict__ acc, int B,
+                                                       int H, int n_q, int n_q_pad, int* __restrict__ dq_sem) {
+  const int64_t rows = (int64_t)B * n_q * H;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t < rows) {
-    const int h = (int)(t % p.H);
-    const int64_t bi = t / p.H;
-    const int i = (int)(bi % p.n_q), b = (int)(bi / p.n_q);
+    const int h = (int)(t % H);
+    const int64_t bi = t / H;
+    const int i = (int)(bi % n_q), b = (int)(bi / n_q);
     float s = 0.f;
     if constexpr (F32) {
-      const float4* po = reinterpret_cast<const float4*>(static_cast<const float*>(p.o) + t * D);
-      const float4* pd = reinterpret_cast<const float4*>(static_cast<const float*>(p.dout) + t * D);
+      const float4* po = reinterpret_cast<const float4*>(static_cast<const float*>(o) + t * D);
+      const float4* pd = reinterpret_cast<const float4*>(static_cast<const float*>(dout) + t * D);
 #pragma unroll 4
       for (int c = 0; c < D / 4; ++c) {
         const float4 a = __ldg(po + c), g = __ldg(pd + c);
         s = fmaf(a.x, g.x, fmaf(a.y, g.y, fmaf(a.z, g.z, fmaf(a.w, g.w, s))));
       }
     } else {
-      const uint4* po = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + t * D);
-      const uint4* pd = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dout) + t * D);
+      const uint4* po = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + t * D);
+      const uint4* pd = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dout) + t * D);
 #pragma unroll 4
       for (int c = 0; c < D / 8; ++c) {
         const uint4 a = __ldg(po + c), g = __ldg(pd + c);
@@ -746,32 +657,26 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const PrepParams p) {
         }
       }
     }
-    const int64_t out = ((int64_t)b * p.H + h) * p.n_q_pad + i;  // rows padded to whole query tiles
-    p.dvec[out] = s;
-    const float l = p.lse[((int64_t)b * p.H + h) * p.n_q + i];
-    p.lse2[out] = (l == kNegInf) ? kPosInf : l * 1.4426950408889634f;
-    const int64_t bhm = (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : h);
-    if (__ldg(p.row_count + bhm * p.T_q + i / kTile) == 0) {  // no contributor: dQ row = 0
-      if constexpr (F32) {
-        float4* row = reinterpret_cast<float4*>(static_cast<float*>(p.dq) + t * D);
-        for (int c = 0; c < D / 4; ++c) row[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        uint4* row = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) + t * D);
-        for (int c = 0; c < D / 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
+    const int64_t out = ((int64_t)b * H + h) * n_q_pad + i;  // rows padded to whole query tiles
+    dvec[out] = s;
+    const float l = lse[((int64_t)b * H + h) * n_q + i];
+    lse2[out] = (l == kNegInf) ? kPosInf : l * 1.4426950408889634f;
   }
   // padding rows past a ragged n_q: P = 0 there (log2 LSE = +inf), D_i = 0
-  const int pad = p.n_q_pad - p.n_q;
+  const int pad = n_q_pad - n_q;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   if (pad > 0)
-    for (int64_t k = t; k < (int64_t)p.B * p.H * pad; k += stride) {
-      const int64_t row = (k / pad) * p.n_q_pad + p.n_q + (k % pad);
-      p.lse2[row] = kPosInf;
-      p.dvec[row] = 0.f;
+    for (int64_t k = t; k < (int64_t)B * H * pad; k += stride) {
+      const int64_t row = (k / pad) * n_q_pad + n_q + (k % pad);
+      lse2[row] = kPosInf;
+      dvec[row] = 0.f;
     }
-  // no key tile has reached any query tile yet
-  for (int64_t k = t; k < 2 * (int64_t)p.B * p.H * p.T_q; k += stride) p.counters[k] = 0;
+  // clear the accumulator (B*H*n_q_pad*D floats), grid-stride in float4
+  float4* a4 = reinterpret_cast<float4*>(acc);
+  const int64_t n4 = (int64_t)B * H * n_q_pad * D / 4;
+  for (int64_t k = t; k < n4; k += stride) a4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (dq_sem)  // fixed-order dQ: no key tile has added yet
+    for (int64_t k = t; k < (int64_t)B * H * (n_q_pad / kTile); k += stride) dq_sem[k] = 0;
 }
 
 // Fixed-order dQ: turn[bhm, kt, qt] = position of key tile kt in the row list of query tile qt
@@ -791,15 +696,53 @@ __global__ void __launch_bounds__(256) bwd_turn_kernel(const int32_t* __restrict
     turn[(bhm * T_k + (__ldg(e + pos) >> 1)) * T_q + qt] = (uint16_t)pos;
 }
 
+// dQ[b, i, h, :] = scale * acc for one 64-row block per CTA: the block (a
+// contiguous 16 x D x 4 fp32 run) is read coalesced into shared memory (padded
+// against bank conflicts), then each thread writes 8 consecutive d of one row.
+template <int D, bool F32>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, void* __restrict__ dq,
+                                                     int B, int H, int n_q, int n_q_pad, float scale) {
+  __shared__ float4 buf[16 * D + 2 * D];  // one float4 of padding per 8
+  const int blocks_per_bh = n_q_pad / 64;
+  const int64_t bh = blockIdx.x / blocks_per_bh;
+  const int qb = blockIdx.x % blocks_per_bh;
+  const int b = (int)(bh / H), h = (int)(bh % H);
+  const float4* src = reinterpret_cast<const float4*>(acc + (bh * n_q_pad + (int64_t)qb * 64) * D);
+  for (int k = threadIdx.x; k < 16 * D; k += blockDim.x) buf[k + (k >> 3)] = __ldg(src + k);
+  __syncthreads();
+  for (int w = threadIdx.x; w < 64 * (D / 8); w += blockDim.x) {
+    const int q = w / (D / 8), d0 = (w % (D / 8)) * 8;
+    if (qb * 64 + q >= n_q) continue;  // padding rows past a ragged n_q
+    const int g = q >> 2, u = q & 3;
+    float x[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int k = g * D + d0 + c;
+      const float4 f = buf[k + (k >> 3)];
+      x[c] = (u == 0 ? f.x : u == 1 ? f.y : u == 2 ? f.z : f.w) * scale;
+    }
+    const int64_t off = (((int64_t)b * n_q + (int64_t)qb * 64 + q) * H + h) * D + d0;
+    if constexpr (F32) {
+      float* row = static_cast<float*>(dq) + off;
+      st_global_v4(row, __float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+      st_global_v4(row + 4, __float_as_uint(x[4]), __float_as_uint(x[5]), __float_as_uint(x[6]),
+                   __float_as_uint(x[7]));
+    } else {
+      __nv_bfloat16* row = static_cast<__nv_bfloat16*>(dq) + off;
+      st_global_v4(row, pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    }
+  }
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct BwdLayout {
-  size_t acc, lse2, dvec, counters, turn, total;
+  size_t acc, lse2, dvec, turn, sem, total;
 };
 
-// Workspace: fp32 dQ accumulator, log2 LSE and D_i per padded row, two int32 counters per query
-// tile (arrival tickets, completed contributors); for fixed-order dQ also the turn table (sized
-// for Hm = H, the larger of the two mask-head counts).
+// Workspace: fp32 dQ accumulator, log2 LSE and D_i per padded row; for fixed-order dQ also the
+// turn table (sized for Hm = H, the larger of the two mask-head counts) and one counter per
+// query tile.
 BwdLayout bwd_layout(const fm_attn_args* a) {
   BwdLayout L;
   const size_t T_q = ((size_t)a->n_q + kTile - 1) / kTile, T_k = ((size_t)a->n_k + kTile - 1) / kTile;
@@ -807,9 +750,11 @@ BwdLayout bwd_layout(const fm_attn_args* a) {
   L.acc = 0;
   L.lse2 = align256(rows * a->D * 4);
   L.dvec = L.lse2 + align256(rows * 4);
-  L.counters = L.dvec + align256(rows * 4);
-  L.turn = L.total = L.counters + align256(2 * (size_t)a->B * a->H * T_q * 4);
-  if (a->deterministic) L.total = L.turn + align256((size_t)a->B * a->H * T_k * T_q * 2);
+  L.turn = L.sem = L.total = L.dvec + align256(rows * 4);
+  if (a->deterministic) {
+    L.sem = L.turn + align256((size_t)a->B * a->H * T_k * T_q * 2);
+    L.total = L.sem + align256((size_t)a->B * a->H * T_q * 4);
+  }
   return L;
 }
 
@@ -824,7 +769,7 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
   float* lse2 = reinterpret_cast<float*>(w + L.lse2);
   float* dvec = reinterpret_cast<float*>(w + L.dvec);
   uint16_t* turn = a->deterministic ? reinterpret_cast<uint16_t*>(w + L.turn) : nullptr;
-  int* counters = reinterpret_cast<int*>(w + L.counters);
+  int* dq_sem = a->deterministic ? reinterpret_cast<int*>(w + L.sem) : nullptr;
   const int H_kv = a->H_kv ? a->H_kv : a->H;
   CUtensorMap tq, tdo, tk, tv, tdk, tdv;
   auto enc = F32 ? encode_tmap_f32_4d : encode_tmap_bf16_4d;
@@ -832,33 +777,15 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
       !enc(&tk, a->k, D, H_kv, a->n_k, a->B, kTile) || !enc(&tv, a->v, D, H_kv, a->n_k, a->B, kTile) ||
       !enc(&tdk, dk, D, H_kv, a->n_k, a->B, kTile) || !enc(&tdv, dv, D, H_kv, a->n_k, a->B, kTile))
     return FM_ERR_CUDA;
-  const int T_q = (a->n_q + kTile - 1) / kTile;
-  PrepParams pp;
-  pp.o = o;
-  pp.dout = dout;
-  pp.lse = lse;
-  pp.lse2 = lse2;
-  pp.dvec = dvec;
-  pp.counters = counters;
-  pp.row_count = meta->row_count;
-  pp.dq = dq;
-  pp.B = a->B;
-  pp.H = a->H;
-  pp.Hm = meta->d.Hm;
-  pp.n_q = a->n_q;
-  pp.n_q_pad = T_q * kTile;
-  pp.T_q = T_q;
   const int64_t rows = (int64_t)a->B * a->n_q * a->H;
-  bwd_prep_kernel<D, F32><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(pp);
+  bwd_prep_kernel<D, F32><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(o, dout, lse, lse2, dvec, acc, a->B,
+      a->H, a->n_q, (a->n_q + kTile - 1) / kTile * kTile, dq_sem);
   BwdParams p;
   p.col_count = meta->col_count;
   p.col_entries = meta->col_entries;
   p.order = turn ? nullptr : meta->bwd_order;  // fixed order: key tiles in ascending order
   p.turn = turn;
-  p.row_count = meta->row_count;
-  p.dq_ticket = counters;
-  p.dq_done = counters + (size_t)a->B * a->H * T_q;
-  p.dq = dq;
+  p.dq_sem = dq_sem;
   for (int c = 0; c < 4; ++c) p.vec[c] = vec ? vec[c] : nullptr;
   p.lse2 = lse2;
   p.dvec = dvec;
@@ -887,6 +814,8 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
                                                                     a->B * meta->d.Hm, p.T_q, p.T_k);
   }
   bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H_kv + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
+  bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (p.n_q_pad / 64)), 256, 0, stream>>>(
+      acc, dq, a->B, a->H, a->n_q, p.n_q_pad, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

@@ -517,21 +517,6 @@ __device__ __forceinline__ bool flag_wait_eq(const int* flag, int want, const in
   }
 }
 
-// Bounded wait until *flag >= want (same give-up rules as flag_wait_eq).
-__device__ __forceinline__ bool flag_wait_ge(const int* flag, int want, const int* status,
-                                             const volatile int* abort) {
-  if (ld_acquire_gpu(flag) >= want) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);
-    if (ld_acquire_gpu(flag) >= want) return true;
-    if ((it & 15u) == 0) {
-      if (*abort || (status && *reinterpret_cast<const volatile int*>(status) != 0)) return false;
-      if (globaltimer() - t0 > kTimeoutNs) return false;
-    }
-  }
-}
-
 __device__ __forceinline__ int ld_nc_i32(const int32_t* p) {
   int v;
   asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));

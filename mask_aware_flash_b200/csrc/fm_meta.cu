@@ -169,15 +169,22 @@ __device__ void sort_order(uint32_t* key, const int32_t* cost_a, bool pairs, int
 // class matrix and its row list (key tiles scanned 32 at a time against the key-tile pass's min/max).
 // The CTA that completes a (b, hm) last also writes that (b, hm)'s two dispatch orders.
 __global__ void __launch_bounds__(kRowsThreads) meta_rows_kernel(const MetaParams p) {
+  extern __shared__ int4 mm_smem[];  // this (b, hm)'s min/max, 2 x int4 per key tile (when it fits)
   __shared__ uint32_t key_f[kOrderMax / 2];
   __shared__ uint32_t key_b[kOrderMax];
   __shared__ int last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bhm = blockIdx.y, qt = blockIdx.x * (kRowsThreads / 32) + warp;
   const unsigned below = (1u << lane) - 1u;
+  const int4* mm_g = reinterpret_cast<const int4*>(p.minmax + (int64_t)bhm * p.T_k * 8);
+  const bool staged = p.T_k <= kOrderMax;  // the launch gives 32 B of shared memory per key tile up to 4096
+  if (staged) {
+    for (int k = threadIdx.x; k < 2 * p.T_k; k += blockDim.x) mm_smem[k] = __ldg(mm_g + k);
+    __syncthreads();
+  }
   if (qt < p.T_q) {
     const int64_t r0 = (int64_t)qt * kTile, r1 = (r0 + kTile < p.n_q) ? r0 + kTile : (int64_t)p.n_q;
-    const int4* mm = reinterpret_cast<const int4*>(p.minmax + (int64_t)bhm * p.T_k * 8);
+    const int4* mm = staged ? mm_smem : mm_g;
     uint8_t* cls = p.cls + ((int64_t)bhm * p.T_q + qt) * p.T_k;
     int32_t* ent = p.row_entries + ((int64_t)bhm * p.T_q + qt) * p.T_k;
     int count = 0;
@@ -185,7 +192,7 @@ __global__ void __launch_bounds__(kRowsThreads) meta_rows_kernel(const MetaParam
       const int kt = k0 + lane;
       int c = 0;
       if (kt < p.T_k) {
-        c = classify(__ldg(mm + 2 * kt), __ldg(mm + 2 * kt + 1), r0, r1);
+        c = classify(mm[2 * kt], mm[2 * kt + 1], r0, r1);
         cls[kt] = (uint8_t)c;
       }
       const unsigned keep = __ballot_sync(0xffffffffu, c != 0);
@@ -331,7 +338,10 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t warps_k = (int64_t)p.BHm * p.T_k;
   fm::meta_cols_kernel<<<(unsigned)((warps_k + 7) / 8), 256, 0, s>>>(p);
-  fm::meta_rows_kernel<<<dim3((unsigned)((p.T_q + 31) / 32), (unsigned)p.BHm), fm::kRowsThreads, 0, s>>>(p);
+  // the query-tile pass stages the (b, hm)'s min/max in shared memory (32 B per key tile, <= 128 KiB)
+  const int rows_smem = p.T_k <= fm::kOrderMax ? p.T_k * 32 : 0;
+  if (!fm::smem_opt_in<fm::meta_rows_kernel>(fm::kOrderMax * 32)) return FM_ERR_CUDA;  // + 24 KiB static
+  fm::meta_rows_kernel<<<dim3((unsigned)((p.T_q + 31) / 32), (unsigned)p.BHm), fm::kRowsThreads, rows_smem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

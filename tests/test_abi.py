@@ -148,7 +148,7 @@ def test_bwd_rejects_before_launch(L):
 
 def test_deterministic_flag(L):
     """Fixed-order dQ: the flag is 0 or 1, and its workspace adds the turn table (2 bytes per
-    (b, h, key tile, query tile), 256-aligned); the per-query-tile counters are there in both modes."""
+    (b, h, key tile, query tile)) and one int32 counter per (b, h, query tile), each 256-aligned."""
     vec = fm.VecArray(None, None, None, None)
     p = [ctypes.c_void_p(0x100000 * (t + 1)) for t in range(6)]
     a, m = _attn(L, n_q=384, n_k=640, H=2)
@@ -156,7 +156,7 @@ def test_deterministic_flag(L):
     a.deterministic = 1
     det = L.fm_attn_bwd_workspace_bytes(ctypes.byref(a))
     al = lambda x: (x + 255) // 256 * 256
-    assert det - base == al(1 * 2 * 5 * 3 * 2)
+    assert det - base == al(1 * 2 * 5 * 3 * 2) + al(1 * 2 * 3 * 4)
     assert L.fm_attn_bwd(ctypes.byref(a), ctypes.byref(m), vec, *p, ctypes.c_void_p(0x900000), base, None) == \
         fm.FM_ERR_WORKSPACE  # the deterministic call needs the larger workspace
     a.deterministic = 2

@@ -54,19 +54,21 @@ struct BwdParams {
   int n_q_pad;                 // n_q rounded up to whole query tiles (row stride of lse2, dvec, dq_acc)
   int H_kv, q_per_kv;          // K/V heads; query heads per K/V head (grouped-query attention)
   int group;                   // heads dispatched together
+  int dh0;                     // D = 256: first d column of the half this launch accumulates (0 or 128)
   float scale, scale_log2;
 };
 
 template <int D, bool F32>
 struct BwdSmem {
   static constexpr int kElem = F32 ? 4 : 2;
-  static constexpr int kQStages = F32 ? 2 : 3;       // fp32 tiles are twice as large
-  static constexpr int kDSBufs = F32 ? 1 : 2;
+  // fp32 tiles are twice as large; D = 256 keeps K and V whole (64 KiB each) beside one Q/dO stage
+  static constexpr int kQStages = D == 256 ? 1 : (F32 ? 2 : 3);
+  static constexpr int kDSBufs = (F32 || D == 256) ? 1 : 2;
   // bf16: K, 128 keys x 128 d (the d >= D part kept zero: K^T is a 128-row MMA operand for dQ^T).
   // fp32 (D = 64): K [key][d] in the first half, K^T [d][key] (K-major, four 8 KiB atoms) in the second;
   // V follows, so the 64 rows past the last K^T atom that a 128-row operand reads stay in bounds.
   static constexpr int kK = 0;
-  static constexpr int kKBytes = kTile * 128 * kElem;
+  static constexpr int kKBytes = kTile * (D > 128 ? D : 128) * kElem;
   static constexpr int kV = kK + kKBytes;
   static constexpr int kQStage = kBQ * D * kElem;    // one 64-row sub-tile of Q (or dO)
   static constexpr int kQ = kV + kTile * D * kElem;  // kQStages x Q
@@ -138,6 +140,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr int NDS = S::kDSBufs;
   constexpr int kAtomElems = 128 / S::kElem;  // elements per 128-byte swizzle span
   constexpr int kAtoms = D * S::kElem / 128;   // swizzle-atom columns of a K / V / Q / dO row
+  // d columns this launch accumulates into dK, dV and dQ: all of D, or one half of D = 256 (from p.dh0)
+  constexpr int DH = D > 128 ? 128 : D;
+  constexpr int kAtomsH = DH * S::kElem / 128;
   constexpr int kKStep = F32 ? 8 : 16;         // elements per UMMA K step (32 bytes)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_base_1024(smem_raw);
@@ -266,15 +271,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0 && cnt > 0) {
       // S^T, dP^T: [key][q]; dV, dK: [key][d] with B MN-major; dQ^T: [d][q] with A and B MN-major
       constexpr uint32_t kIdSdp = F32 ? idesc_tf32(128, kBQ, false, false) : idesc_bf16(128, kBQ, false, false);
-      constexpr uint32_t kIdAcc = F32 ? idesc_tf32(128, D, false, true) : idesc_bf16(128, D, false, true);
+      constexpr uint32_t kIdAcc = F32 ? idesc_tf32(128, DH, false, true) : idesc_bf16(128, DH, false, true);
       constexpr uint32_t kIdDq = F32 ? idesc_tf32(128, kBQ, true, true) : idesc_bf16(128, kBQ, true, true);
       // descriptor words (128-byte swizzle, SBO = 8 rows x 128 B); per k-step only the low word moves
       constexpr uint32_t kHi = desc_hi(1024);
       constexpr uint32_t kStageW = S::kQStage >> 4, kDSW = S::kDSBytes >> 4;
       const uint32_t lo_k = desc_lo(k_s, 16), lo_v = desc_lo(v_s, 16);           // K-major A of S^T, dP^T
-      const uint32_t lo_kt = desc_lo(k_s, 16384);                                  // K^T as MN-major A of dQ^T
+      const int ah = (p.dh0 / 64);  // first atom column of this launch's d half (0 unless D = 256)
+      const uint32_t lo_kt = desc_lo(k_s + ah * 16384, 16384);                     // K^T as MN-major A of dQ^T
       const uint32_t lo_q = desc_lo(q_s, 16), lo_do = desc_lo(do_s, 16);         // K-major B of S^T, dP^T
-      const uint32_t lo_qmn = desc_lo(q_s, 8192), lo_domn = desc_lo(do_s, 8192);  // MN-major B of dK, dV
+      const uint32_t lo_qmn = desc_lo(q_s + ah * 8192, 8192), lo_domn = desc_lo(do_s + ah * 8192, 8192);  // B of dK, dV
       const uint32_t lo_ds = desc_lo(ds_s, 16), lo_dsmn = desc_lo(ds_s, 16384);   // dS^T as A of dK / B of dQ^T
       auto issue_s = [&](int i) {  // S^T_i = K Q_i^T
         const uint32_t qa = lo_q + (i % NS) * kStageW, tS = tmem + (i & 1) * 64;
@@ -518,7 +524,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int i = 0; ok && i < nsub; ++i) {
       const int q0 = sub_q0(i);
       const int64_t bh = (int64_t)b * p.H + hq0 + (G > 1 ? head_of(i, jh) : 0);
-      float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q_pad * D;
+      float* acc_bh = p.dq_acc + bh * (int64_t)p.n_q_pad * D + p.dh0 * 4;
       if constexpr (F32) {
         const int st = i % NS;
         ok = all_drain_threads(mbar_wait(bar(S::QT_GO0 + st), (i / NS) & 1, abort_flag));
@@ -540,7 +546,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = all_drain_threads(d != 0 || flag_wait_eq(sem, turn[i >> 1], p.status, abort_flag));
         if (!ok) break;
       }
-      if (d < D) {
+      if (d < DH) {
         float* blk = acc_bh + (int64_t)q0 * D;  // [16 groups of 4 queries][D][4]
 #pragma unroll
         for (int g = 0; g < 16; ++g)
@@ -571,7 +577,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tsrc = (is_dk ? tdK : tdV) + lane_addr;
     uint8_t* stage = smem + (is_dk ? S::kDO : S::kQ);
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
+    for (int cc = 0; cc < DH / 32; ++cc) {
       uint32_t a[32];
       if (have) {
         tmem_ld32(tsrc + cc * 32, a);
@@ -603,8 +609,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fence_proxy_async_smem();
     named_bar_sync(is_dk ? 3 : 2, 128);
     if (r == 0) {
-      for (int c = 0; c < kAtoms; ++c)
-        tma_store_4d(is_dk ? &tm_dk : &tm_dv, smem_u32(stage + c * 16384), c * kAtomElems, hk, kt * kTile, b);
+      for (int c = 0; c < kAtomsH; ++c)
+        tma_store_4d(is_dk ? &tm_dk : &tm_dv, smem_u32(stage + c * 16384), p.dh0 + c * kAtomElems, hk, kt * kTile, b);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -696,40 +702,48 @@ __global__ void __launch_bounds__(256) bwd_turn_kernel(const int32_t* __restrict
     turn[(bhm * T_k + (__ldg(e + pos) >> 1)) * T_q + qt] = (uint16_t)pos;
 }
 
-// dQ[b, i, h, :] = scale * acc for one 64-row block per CTA: the block (a
-// contiguous 16 x D x 4 fp32 run) is read coalesced into shared memory (padded
-// against bank conflicts), then each thread writes 8 consecutive d of one row.
+// dQ[b, i, h, :] = scale * acc for one 64-row block per CTA: the block (16 groups of 4 rows, each
+// D x 4 fp32) is read coalesced into shared memory (padded against bank conflicts) a chunk of at
+// most 128 d columns at a time, then each thread writes 8 consecutive d of one row.
 template <int D, bool F32>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, void* __restrict__ dq,
                                                      int B, int H, int n_q, int n_q_pad, float scale) {
-  __shared__ float4 buf[16 * D + 2 * D];  // one float4 of padding per 8
+  constexpr int DC = D > 128 ? 128 : D;  // d columns per chunk
+  __shared__ float4 buf[16 * DC + 2 * DC];  // one float4 of padding per 8
   const int blocks_per_bh = n_q_pad / 64;
   const int64_t bh = blockIdx.x / blocks_per_bh;
   const int qb = blockIdx.x % blocks_per_bh;
   const int b = (int)(bh / H), h = (int)(bh % H);
   const float4* src = reinterpret_cast<const float4*>(acc + (bh * n_q_pad + (int64_t)qb * 64) * D);
-  for (int k = threadIdx.x; k < 16 * D; k += blockDim.x) buf[k + (k >> 3)] = __ldg(src + k);
-  __syncthreads();
-  for (int w = threadIdx.x; w < 64 * (D / 8); w += blockDim.x) {
-    const int q = w / (D / 8), d0 = (w % (D / 8)) * 8;
-    if (qb * 64 + q >= n_q) continue;  // padding rows past a ragged n_q
-    const int g = q >> 2, u = q & 3;
-    float x[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int k = g * D + d0 + c;
-      const float4 f = buf[k + (k >> 3)];
-      x[c] = (u == 0 ? f.x : u == 1 ? f.y : u == 2 ? f.z : f.w) * scale;
+#pragma unroll 1
+  for (int dc0 = 0; dc0 < D; dc0 += DC) {
+    if (dc0 > 0) __syncthreads();  // the previous chunk's reads of buf are done
+    for (int k = threadIdx.x; k < 16 * DC; k += blockDim.x) {
+      const int g = k / DC, dd = k % DC;
+      buf[k + (k >> 3)] = __ldg(src + g * D + dc0 + dd);
     }
-    const int64_t off = (((int64_t)b * n_q + (int64_t)qb * 64 + q) * H + h) * D + d0;
-    if constexpr (F32) {
-      float* row = static_cast<float*>(dq) + off;
-      st_global_v4(row, __float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
-      st_global_v4(row + 4, __float_as_uint(x[4]), __float_as_uint(x[5]), __float_as_uint(x[6]),
-                   __float_as_uint(x[7]));
-    } else {
-      __nv_bfloat16* row = static_cast<__nv_bfloat16*>(dq) + off;
-      st_global_v4(row, pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    __syncthreads();
+    for (int w = threadIdx.x; w < 64 * (DC / 8); w += blockDim.x) {
+      const int q = w / (DC / 8), d0 = (w % (DC / 8)) * 8;
+      if (qb * 64 + q >= n_q) continue;  // padding rows past a ragged n_q
+      const int g = q >> 2, u = q & 3;
+      float x[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int k = g * DC + d0 + c;
+        const float4 f = buf[k + (k >> 3)];
+        x[c] = (u == 0 ? f.x : u == 1 ? f.y : u == 2 ? f.z : f.w) * scale;
+      }
+      const int64_t off = (((int64_t)b * n_q + (int64_t)qb * 64 + q) * H + h) * D + dc0 + d0;
+      if constexpr (F32) {
+        float* row = static_cast<float*>(dq) + off;
+        st_global_v4(row, __float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+        st_global_v4(row + 4, __float_as_uint(x[4]), __float_as_uint(x[5]), __float_as_uint(x[6]),
+                     __float_as_uint(x[7]));
+      } else {
+        __nv_bfloat16* row = static_cast<__nv_bfloat16*>(dq) + off;
+        st_global_v4(row, pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+      }
     }
   }
 }
@@ -813,7 +827,11 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
     bwd_turn_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(meta->row_count, meta->row_entries, turn,
                                                                     a->B * meta->d.Hm, p.T_q, p.T_k);
   }
-  bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H_kv + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(tq, tdo, tk, tv, tdk, tdv, p);
+  // D = 256: dK, dV and dQ are accumulated one 128-column half per launch (TMEM holds 256 columns of
+  // dK and dV at most); both launches form S^T and dP^T over all 256 columns
+  for (p.dh0 = 0; p.dh0 < D; p.dh0 += (D > 128 ? 128 : D))
+    bwd_kernel<D, F32><<<dim3(p.group * p.T_k, (p.H_kv + p.group - 1) / p.group, p.B), kBwdThreads, S::kAlloc, stream>>>(
+        tq, tdo, tk, tv, tdk, tdv, p);
   bwd_dq_kernel<D, F32><<<(unsigned)((int64_t)a->B * a->H * (p.n_q_pad / 64)), 256, 0, stream>>>(
       acc, dq, a->B, a->H, a->n_q, p.n_q_pad, a->scale);
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
@@ -826,7 +844,7 @@ fm_status launch_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int3
 fm_status check_bwd_args(const fm_attn_args* a, const fm_mask_meta* meta, const int32_t* const vec[4]) {
   const fm_status st = check_attn_args(a, meta, vec);
   if (st != FM_OK) return st;
-  if (a->D == 256) return FM_ERR_UNSUPPORTED;  // the backward takes D in {64, 128}
+  if (a->D == 256 && a->deterministic) return FM_ERR_UNSUPPORTED;  // fixed-order dQ: D in {64, 128}
   const int H_kv = a->H_kv ? a->H_kv : a->H;
   if ((int64_t)(a->H / H_kv) * ((a->n_q + 127) / 128) > kMaxList) return FM_ERR_UNSUPPORTED;
   return FM_OK;
@@ -837,7 +855,7 @@ fm_status check_bwd_args(const fm_attn_args* a, const fm_mask_meta* meta, const 
 extern "C" {
 
 size_t fm_attn_bwd_workspace_bytes(const fm_attn_args* a) {
-  if (!a || a->B < 1 || a->H < 1 || a->n_q < 1 || (a->D != 64 && a->D != 128)) return 0;
+  if (!a || a->B < 1 || a->H < 1 || a->n_q < 1 || (a->D != 64 && a->D != 128 && a->D != 256)) return 0;
   return fm::bwd_layout(a).total;
 }
 
@@ -855,6 +873,7 @@ fm_status fm_attn_bwd(const fm_attn_args* a, const fm_mask_meta* meta, const int
     return FM_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (a->dtype == 1) return fm::launch_bwd<64, true>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s);
+  if (a->D == 256) return fm::launch_bwd<256, false>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s);
   return a->D == 64 ? fm::launch_bwd<64, false>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s)
                     : fm::launch_bwd<128, false>(a, meta, vec, o, lse, dout, dq, dk, dv, ws, s);
 }

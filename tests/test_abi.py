@@ -239,3 +239,17 @@ def test_noalloc_rejects_oversize(L):
     p = [ctypes.c_void_p(0x100000 * (t + 1)) for t in range(6)]
     rc = L.fm_attn_bwd_noalloc(ctypes.byref(a), ctypes.byref(m), fm.VecArray(None, None, None, None), *p, None)
     assert rc == fm.FM_ERR_WORKSPACE
+
+
+@pytest.mark.skipif(torch_cuda_present(), reason="hands made-up device addresses to an entry point that can launch")
+def test_head_dim_256_fixed_order_rejected(L):
+    """D = 256 runs the backward in two launches over the two halves of d; the fixed-order dQ mode is
+    not offered there: FM_ERR_UNSUPPORTED on the host."""
+    vec = fm.VecArray(None, None, None, None)
+    p = [ctypes.c_void_p(0x100000 * (t + 1)) for t in range(6)]
+    a, m = _attn(L, n_q=384, n_k=640, H=2)
+    a.D = 256
+    a.deterministic = 1
+    assert L.fm_attn_bwd_workspace_bytes(ctypes.byref(a)) > 0
+    assert L.fm_attn_bwd(ctypes.byref(a), ctypes.byref(m), vec, *p, ctypes.c_void_p(0x900000), 1 << 30, None) == \
+        fm.FM_ERR_UNSUPPORTED

@@ -265,6 +265,16 @@ def test_head_dim_256_forward(fm, n, family):
     _compare(res, vecs, 1, bwd=False)
 
 
+@pytest.mark.parametrize("n,family", [(256, "causal_document"), (640, "full"), (1000, "random_eviction"),
+                                      (388, "share_question"), (1536, "global_sliding")])
+def test_head_dim_256_backward(fm, n, family):
+    """D = 256 backward (dK, dV and dQ accumulated one 128-column half per launch, S^T and dP^T over
+    all 256 columns in both): every row and column of both heads against the oracle."""
+    vecs = _vec_stack(synth.make_family(family, n, 73), 1, 1)
+    res = _run_attention(fm, 1, 2, n, n, 256, vecs, 1, seed=74)
+    _compare(res, vecs, 1)
+
+
 def _run_fp32(fm, B, H, n, vecs, seed):
     """fp32 inputs and outputs (tf32 tensor-core products), D = 64."""
     D = 64

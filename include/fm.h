@@ -57,7 +57,9 @@ typedef enum {
   FM_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. n_k not a multiple of 4) */
   FM_ERR_WORKSPACE = 3,       /* workspace pointer NULL/misaligned or ws_bytes too small */
   FM_ERR_CUDA = 4,            /* a CUDA runtime/driver call or launch failed */
-  FM_ERR_DEVICE_TIMEOUT = 5   /* a kernel's bounded wait ran out (see fm_get_device_status) */
+  FM_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (see fm_get_device_status) */
+  FM_ERR_DEVICE_CHECK = 6     /* FM_DEBUG builds only: an index or shared-memory canary check failed on
+                                 the device (the access was skipped; see fm_get_device_status) */
 } fm_status;
 
 /* Shape of a mask problem.  tile_q and tile_k must be 128. */

@@ -22,10 +22,13 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfm_b200.so")
+# FM_DEBUG=1 in the environment loads the checking build (device-side index checks and shared-memory
+# canaries; failures come back as FM_ERR_DEVICE_CHECK from fm_get_device_status)
+LIB_PATH = os.path.join(_HERE, "libfm_b200_debug.so" if os.environ.get("FM_DEBUG") == "1" else "libfm_b200.so")
 _lib = None
 
-FM_OK, FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA, FM_ERR_DEVICE_TIMEOUT = range(6)
+FM_OK, FM_ERR_INVALID_ARG, FM_ERR_UNSUPPORTED, FM_ERR_WORKSPACE, FM_ERR_CUDA, FM_ERR_DEVICE_TIMEOUT, \
+    FM_ERR_DEVICE_CHECK = range(7)
 TILE = 128
 META_LAUNCHES = 2  # kernels one fm_build_mask_meta call launches
 BWD_LAUNCHES = 3   # kernels one fm_attn_bwd call launches (one more with deterministic=True)

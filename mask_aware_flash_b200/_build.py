@@ -13,6 +13,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libfm_b200.so")
+# FM_DEBUG variant: device-side index checks and shared-memory canaries (see fm_common.cuh)
+LIB_DEBUG = os.path.join(HERE, "libfm_b200_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -32,20 +34,22 @@ def deps():
         os.path.join(ROOT, "include", "fm.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [NVCC] + FLAGS + ["-I", os.path.join(ROOT, "include")]
+def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False, debug: bool = False) -> str:
+    """Compile csrc/*.cu into libfm_b200.so (debug=True: libfm_b200_debug.so with -DFM_DEBUG)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    cmd = [NVCC] + FLAGS + ["-I", os.path.join(ROOT, "include")] + (["-DFM_DEBUG"] if debug else [])
     if ptxas_v:
         cmd += ["-Xptxas", "-v"]
-    cmd += sources() + ["-o", LIB]
+    cmd += sources() + ["-o", lib]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -53,8 +57,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> 
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose or ptxas_v:
         sys.stderr.write(r.stdout + r.stderr)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, verbose=True, ptxas_v="-v" in sys.argv)
+    build(force=True, verbose=True, ptxas_v="-v" in sys.argv, debug="--debug" in sys.argv)

@@ -114,6 +114,7 @@ const char* fm_status_string(fm_status s) {
     case FM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case FM_ERR_CUDA: return "CUDA call or kernel launch failed";
     case FM_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out on the device";
+    case FM_ERR_DEVICE_CHECK: return "a device-side index or canary check failed (debug build)";
   }
   return "unknown status";
 }

@@ -85,7 +85,8 @@ struct BwdSmem {
          QT_GO0, QT_GO1, QT_READY0, QT_READY1, KT_READY,  // fp32 path: operand transposes
          kNumBars };
   static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort, [2] zero flag
-  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kCanaryAt = kMisc + 16;        // FM_DEBUG: shared-memory canary words
+  static constexpr int kBytes = kCanaryAt + kCanaryBytes;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -158,8 +159,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int G = p.q_per_kv, hq0 = hk * G;
   auto bhm_of = [&](int hq) -> int64_t { return (int64_t)b * p.Hm + (p.Hm == 1 ? 0 : hq); };
   const int kt = p.order ? __ldg(p.order + bhm_of(hq0) * p.T_k + blockIdx.x / p.group) : (int)(blockIdx.x / p.group);
-  int cnt = 0;  // entries over the group's query heads
-  for (int jq = 0; jq < G; ++jq) cnt += __ldg(p.col_count + bhm_of(hq0 + jq) * p.T_k + kt);
+  int cnt_raw = 0;  // entries over the group's query heads
+  for (int jq = 0; jq < G; ++jq) cnt_raw += __ldg(p.col_count + bhm_of(hq0 + jq) * p.T_k + kt);
+  const int cnt = kDebug ? min(max(cnt_raw, 0), kMaxList) : cnt_raw;  // (debug: recorded below, clamped)
   const int nsub = 2 * cnt;  // two 64-row sub-tiles per listed 128-row query tile
 
   const uint32_t bar0 = smem_u32(smem + S::kBar);
@@ -182,6 +184,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(S::KT_READY), kTile);
     *abort_flag = 0;
     misc[2] = 0;
+    canary_write(smem + S::kCanaryAt);
+    check_range(cnt_raw, 0, kMaxList + 1, p.status, abort_flag, 51);
     fence_barrier_init();
     {  // K and V first (as soon as the key tile is known): their latency overlaps the list copy and
        // the TMEM allocation.  A CTA with an empty list waits for them before it exits.
@@ -208,10 +212,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int cj = __ldg(p.col_count + bj * p.T_k + kt);
       const int32_t* ej = p.col_entries + (bj * p.T_k + kt) * p.T_q;
       if (threadIdx.x == 0) hstart[jq] = start;
-      for (int t = threadIdx.x; t < cj; t += kBwdThreads) {
+      const int cj_room = kDebug ? min(cj, cnt - start) : cj;  // (debug: never past the clamped total)
+      for (int t = threadIdx.x; t < cj_room; t += kBwdThreads) {
         const int32_t e = __ldg(ej + (rev ? cj - 1 - t : t));
         list[start + t] = (uint16_t)e;
-        if (rev) turn[start + t] = __ldg(p.turn + (bj * p.T_k + kt) * p.T_q + (e >> 1));
+        if (rev && (!kDebug || (e >> 1) < p.T_q)) turn[start + t] = __ldg(p.turn + (bj * p.T_k + kt) * p.T_q + (e >> 1));
       }
       start += cj;
     }
@@ -254,6 +259,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         const int q0 = sub_q0(i);
+        if (!check_range(q0 >> 7, 0, p.T_q, p.status, abort_flag, 52)) break;  // a list entry past the query tiles
         const int hq = hq0 + (G > 1 ? head_of(i, jh) : 0);
         const int64_t bh = (int64_t)b * p.H + hq;
         const uint32_t fb = bar(S::QDO_FULL0 + st);
@@ -311,23 +317,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_commit(bar(S::SDP_FULL));
         if constexpr (F32) umma_commit(bar(S::QT_GO0));
       }
+      // next sub-tile's S^T (other buffer) and dP^T.  With two or more Q/dO stages they are issued
+      // before this sub-tile's dV / dK / dQ^T, so they overlap its softmax; with one stage (D = 256) the
+      // next Q/dO can only arrive once this sub-tile's dV and dK have read the stage, so they follow.
+      auto issue_next = [&](int i) -> bool {
+        if (i + 1 >= nsub) return true;
+        if (!mbar_wait(bar(S::QDO_FULL0 + (i + 1) % NS), ((i + 1) / NS) & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_s(i + 1);
+        if (!mbar_wait(bar(S::DP_FREE), i & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_dp(i + 1);
+        umma_commit(bar(S::SDP_FULL));
+        if constexpr (F32) umma_commit(bar(S::QT_GO0 + (i + 1) % NS));
+        return true;
+      };
       for (int i = 0; ok && i < nsub; ++i) {
         const int st = i % NS, bi = i % NDS;
-        if (i + 1 < nsub) {  // next sub-tile's S^T (other buffer) and dP^T, overlapping this sub-tile's softmax
-          if (!mbar_wait(bar(S::QDO_FULL0 + (i + 1) % NS), ((i + 1) / NS) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_s(i + 1);
-          if (!mbar_wait(bar(S::DP_FREE), i & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_dp(i + 1);
-          umma_commit(bar(S::SDP_FULL));
-          if constexpr (F32) umma_commit(bar(S::QT_GO0 + (i + 1) % NS));
+        if (NS > 1 && !issue_next(i)) {
+          ok = false;
+          break;
         }
         if (!mbar_wait(bar(S::DS_READY), i & 1, abort_flag)) {
           ok = false;
@@ -389,6 +398,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         umma_commit(bar(S::DQ_FULL));
         umma_commit(bar(S::DS_EMPTY0 + bi));
+        if (NS == 1 && !issue_next(i)) ok = false;
       }
       if (!ok) record_failure(p.status, abort_flag, 12);
       umma_commit(bar(S::ACC_FULL));
@@ -546,7 +556,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = all_drain_threads(d != 0 || flag_wait_eq(sem, turn[i >> 1], p.status, abort_flag));
         if (!ok) break;
       }
-      if (d < DH) {
+      if (d < DH && (!kDebug || check_range(q0 >> 7, 0, p.T_q, p.status, abort_flag, 53))) {
         float* blk = acc_bh + (int64_t)q0 * D;  // [16 groups of 4 queries][D][4]
 #pragma unroll
         for (int g = 0; g < 16; ++g)
@@ -619,6 +629,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0 && cnt == 0) mbar_wait(bar(S::KV_FULL), 0, never);  // no copy in flight at exit
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) canary_check(smem + S::kCanaryAt, p.status, abort_flag, 54);
   if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -79,6 +79,42 @@ __device__ __forceinline__ void record_failure(int* status, volatile int* abort,
 }
 
 // ---------------------------------------------------------------------------
+// FM_DEBUG builds: device-side checks that stand in for a sanitizer.  A failed check latches
+// FM_ERR_DEVICE_CHECK (with the site and the offending value's low bits) into the status word,
+// raises the CTA abort flag (so every role stops waiting and unwinds), and the access is skipped.
+// Shared-memory canaries: each kernel writes kCanary words just past its layout at entry and
+// checks them at exit.  Without FM_DEBUG every check compiles to nothing.
+// ---------------------------------------------------------------------------
+#ifdef FM_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
+constexpr uint32_t kCanary = 0xFEEDC0DEu;
+constexpr int kCanaryBytes = 16;
+
+__device__ __forceinline__ void record_check(int* status, volatile int* abort, int site, int value) {
+  *abort = 1;
+  if (status) atomicCAS(status, 0, (FM_ERR_DEVICE_CHECK << 16) | ((site & 0xFF) << 8) | (value & 0xFF));
+}
+// true if lo <= v < hi; otherwise (debug builds) records the failure and returns false
+__device__ __forceinline__ bool check_range(int v, int lo, int hi, int* status, volatile int* abort, int site) {
+  if constexpr (!kDebug) return true;
+  if (v >= lo && v < hi) return true;
+  record_check(status, abort, site, v);
+  return false;
+}
+__device__ __forceinline__ void canary_write(uint8_t* p) {
+  if constexpr (kDebug)
+    for (int k = 0; k < kCanaryBytes / 4; ++k) reinterpret_cast<volatile uint32_t*>(p)[k] = kCanary ^ k;
+}
+__device__ __forceinline__ void canary_check(const uint8_t* p, int* status, volatile int* abort, int site) {
+  if constexpr (kDebug)
+    for (int k = 0; k < kCanaryBytes / 4; ++k)
+      if (reinterpret_cast<const volatile uint32_t*>(p)[k] != (kCanary ^ k)) record_check(status, abort, site, k);
+}
+
+// ---------------------------------------------------------------------------
 // TMA and bulk copies (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,

@@ -68,7 +68,8 @@ struct FwdSmem {
          P_FULL0, P_FULL1, P_HALF0, P_HALF1, O_DONE0, O_DONE1, M_FULL0, M_FULL1, M_EMPTY0, M_EMPTY1, DRAIN,
          kNumBars };
   static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag, [2] zero
-  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kCanaryAt = kMisc + 16;        // FM_DEBUG: shared-memory canary words
+  static constexpr int kBytes = kCanaryAt + kCanaryBytes;
   static constexpr int kAlloc = kBytes + 1024;       // slack for 1024-byte alignment of the base
 };
 
@@ -143,8 +144,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const bool has1 = qt1 < p.T_q;
   const int32_t* rows0 = p.row_entries + (bhm * p.T_q + qt0) * p.T_k;
   const int32_t* rows1 = rows0 + p.T_k;
-  const int n0 = __ldg(p.row_count + bhm * p.T_q + qt0);
-  const int n1 = has1 ? __ldg(p.row_count + bhm * p.T_q + qt1) : 0;
+  const int n0_raw = __ldg(p.row_count + bhm * p.T_q + qt0);
+  const int n1_raw = has1 ? __ldg(p.row_count + bhm * p.T_q + qt1) : 0;
+  // (debug builds: a count beyond the shared-memory list is recorded below and clamped)
+  const int n0 = kDebug ? min(max(n0_raw, 0), kMaxList) : n0_raw;
+  const int n1 = kDebug ? min(max(n1_raw, 0), kMaxList) : n1_raw;
   const int ragged_kt = (p.n_k % kTile) ? p.T_k - 1 : -1;
 
   const uint32_t bar0 = smem_u32(smem + S::kBar);
@@ -167,6 +171,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(bar(S::M_EMPTY1), 2 * kTile);
     *abort_flag = 0;
     misc[2] = 0;  // a flag nothing raises: lets the final drain wait ignore aborts
+    canary_write(smem + S::kCanaryAt);
+    check_range(n0_raw, 0, kMaxList + 1, p.status, abort_flag, 31);
+    check_range(n1_raw, 0, kMaxList + 1, p.status, abort_flag, 32);
     fence_barrier_init();
     if (n0 + n1 > 0) {  // Q first: its latency overlaps the list copy and the TMEM allocation
       fence_proxy_async_smem();
@@ -214,6 +221,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = true;
       while (it.next(kt, c0, c1)) {
         const int slot = e & 1;
+        if (!check_range(kt, 0, p.T_k, p.status, abort_flag, 33)) {  // a list entry past the key tiles
+          ok = false;
+          break;
+        }
         if (e >= 2 && !wait_all(bar(S::K_EMPTY0 + slot), ((e >> 1) - 1) & 1)) {
           ok = false;
           break;
@@ -569,6 +580,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) canary_check(smem + S::kCanaryAt, p.status, abort_flag, 34);
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -599,7 +611,8 @@ struct Fwd256Smem {
   enum { Q_FULL, K_FULL0, K_FULL1, K_EMPTY0, K_EMPTY1, V_FULL0, V_FULL1, V_EMPTY0, V_EMPTY1, S_FULL0, S_FULL1,
          P_HALF0, P_HALF1, P_FULL0, P_FULL1, O_DONE, M_FULL0, M_FULL1, M_EMPTY0, M_EMPTY1, DRAIN, kNumBars };
   static constexpr int kMisc = kBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag, [2] zero
-  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kCanaryAt = kMisc + 16;        // FM_DEBUG: shared-memory canary words
+  static constexpr int kBytes = kCanaryAt + kCanaryBytes;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -621,7 +634,8 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
   const int qt = 2 * __ldg(p.order + bhm * p.n_pairs + rank / 2) + (rank & 1);
   if (qt >= p.T_q) return;  // odd tile count: the pair's second tile does not exist
   const int32_t* rows = p.row_entries + (bhm * p.T_q + qt) * p.T_k;
-  const int n = __ldg(p.row_count + bhm * p.T_q + qt);
+  const int n_raw = __ldg(p.row_count + bhm * p.T_q + qt);
+  const int n = kDebug ? min(max(n_raw, 0), kMaxList) : n_raw;  // (debug: recorded below, clamped)
   const int ragged_kt = (p.n_k % kTile) ? p.T_k - 1 : -1;
 
   const uint32_t bar0 = smem_u32(smem + S::kBar);
@@ -643,6 +657,8 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
     mbar_init(bar(S::M_EMPTY1), kTile);
     *abort_flag = 0;
     misc[2] = 0;
+    canary_write(smem + S::kCanaryAt);
+    check_range(n_raw, 0, kMaxList + 1, p.status, abort_flag, 41);
     fence_barrier_init();
     if (n > 0) {
       fence_proxy_async_smem();
@@ -679,6 +695,10 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
       for (int e = 0; ok && e < n; ++e) {
         int kt;
         const int c = cls_of(e, kt);
+        if (!check_range(kt, 0, p.T_k, p.status, abort_flag, 42)) {  // a list entry past the key tiles
+          ok = false;
+          break;
+        }
         for (int hh = 0; hh < 2; ++hh) {
           const int u = 2 * e + hh, slot = u & 1;
           if (u >= 2 && !mbar_wait(bar(S::K_EMPTY0 + slot), ((u >> 1) - 1) & 1, abort_flag)) {
@@ -940,6 +960,7 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) canary_check(smem + S::kCanaryAt, p.status, abort_flag, 43);
   if (warp == 6) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

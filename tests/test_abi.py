@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(6):
+    for code in range(7):
         assert fm.status_string(code) and fm.status_string(code) != "unknown status"
     assert fm.status_string(99) == "unknown status"
 

@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="n131072", choices=["n131072", "n32768", "n8192"])
     ap.add_argument("--masks", default=None, help="comma list of mask names (default: the config's)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the config's head count (small ncu captures; the bench line then names it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the phases eagerly instead of graph replays")
@@ -59,7 +61,7 @@ def parse():
 
 
 # ----------------------------------------------------------------------------- workload
-def workload(config: str, rank: int, masks_arg=None):
+def workload(config: str, rank: int, masks_arg=None, heads=None):
     if config == "n8192":
         n, B, H, D = 8192, 2, 16, 128
         masks = ["sliding_window_1024", "causal_document_512_4096"]
@@ -77,6 +79,9 @@ def workload(config: str, rank: int, masks_arg=None):
     if masks_arg:
         masks = masks_arg.split(",")
         desc = desc.split(";")[0] + "; masks: " + ", ".join(masks)
+    if heads:
+        desc = desc.replace(f"H={H} ", f"H={heads} ", 1)
+        H = heads
     cfg_id = {"n8192": 2, "n32768": 3, "n131072": 4}[config]
     specs = []
     for m_idx, name in enumerate(masks):
@@ -297,7 +302,7 @@ def run_ours(args, rank, world, local_rank):
     _build.build()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = workload(args.config, rank, args.masks)
+    wl = workload(args.config, rank, args.masks, args.heads)
     n, B, H, D = wl["n"], wl["B"], wl["H"], wl["D"]
     scale = 1.0 / math.sqrt(D)
 
@@ -668,7 +673,7 @@ def aux_meta(fm, torch, dev, stream, hbm, reps):
 
 
 def run_reference(args):
-    wl = workload(args.config, 0, args.masks)
+    wl = workload(args.config, 0, args.masks, args.heads)
     cb = cpu_baseline(wl, budget_s=max(5.0, min(20.0, 3.0 * args.steps)))
     return {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",

@@ -217,23 +217,29 @@ def peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def lib_hash():
+KERNEL_SOURCES = {  # the files whose device code each timed kernel is built from
+    "bwd_kernel": ["mask_aware_flash_b200/csrc/fm_bwd.cu", "mask_aware_flash_b200/csrc/fm_common.cuh", "include/fm.h"],
+    "fwd_kernel": ["mask_aware_flash_b200/csrc/fm_fwd.cu", "mask_aware_flash_b200/csrc/fm_common.cuh", "include/fm.h"],
+}
+
+
+def source_hash(kernel: str) -> str:
+    """Hash of the sources a kernel is built from (a committed traffic figure is valid for it)."""
     h = hashlib.sha256()
-    for d in ("mask_aware_flash_b200/csrc",):
-        for f in sorted(os.listdir(os.path.join(ROOT, d))):
-            with open(os.path.join(ROOT, d, f), "rb") as fh:
-                h.update(fh.read())
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel: str, config: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current sources."""
+    """DRAM bytes per launch from a committed ncu summary, if it matches the kernel's current sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
         e = t[config][kernel]
-        return e["bytes_per_launch"] if e.get("source_hash") == lib_hash() else None
+        return e["bytes_per_launch"] if e.get("source_hash") == source_hash(kernel) else None
     except Exception:
         return None
 

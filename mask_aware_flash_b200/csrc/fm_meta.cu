@@ -14,10 +14,10 @@ namespace fm {
 namespace {
 
 constexpr int kTile = 128;
+constexpr int kOrderListMax = 4096;  // longest list (tiles each way) the attention kernels take
 
 struct MetaParams {
   const int32_t* vec[4];  // [B, Hm, n_k] or null
-  bool vec16;             // every vector row starts 16-byte aligned (n_k % 4 == 0): 16-byte loads
   int32_t* minmax;        // [BHm, T_k, 8]
   uint8_t* cls;           // [BHm, T_q, T_k]
   int32_t* row_count;     // [BHm, T_q]
@@ -34,92 +34,143 @@ __device__ __forceinline__ int32_t vec_at(const int32_t* v, int64_t idx, int32_t
   return v ? __ldg(v + idx) : dflt;
 }
 
+// Last row (exclusive) of the tile starting at row r0: min(r0 + 128, n_q), without overflow.
+__device__ __forceinline__ int tile_r1(int r0, int n_q) { return (n_q - r0 > kTile) ? r0 + kTile : n_q; }
+
 // 0 skip, 1 partial, 2 full for query rows [r0, r1) against one key tile's min/max.
-__device__ __forceinline__ int classify(const int4 lo, const int4 hi, int64_t r0, int64_t r1) {
+__device__ __forceinline__ int classify(const int4 lo, const int4 hi, int r0, int r1) {
   // lo = (minLTS, maxLTS, minLTE, maxLTE), hi = (minUTS, maxUTS, minUTE, maxUTE)
-  const bool skip = ((int64_t)lo.y <= r0 && (int64_t)lo.z >= r1) || ((int64_t)hi.y <= r0 && (int64_t)hi.z >= r1);
-  const bool clear_l = ((int64_t)lo.x >= r1) || ((int64_t)lo.w <= r0);
-  const bool clear_u = ((int64_t)hi.x >= r1) || ((int64_t)hi.w <= r0);
+  const bool skip = (lo.y <= r0 && lo.z >= r1) || (hi.y <= r0 && hi.z >= r1);
+  const bool clear_l = (lo.x >= r1) || (lo.w <= r0);
+  const bool clear_u = (hi.x >= r1) || (hi.w <= r0);
   return skip ? 0 : ((clear_l && clear_u) ? 2 : 1);
 }
 
-// Key-tile pass: one warp per (bhm, key tile).  Min and max of the four vectors over the tile's 128
-// columns (one 16-byte load per lane and vector when the rows are 16-byte aligned), written to
-// minmax, then the tile's column list: every query tile classified against those eight values,
-// 32 per step, the non-skip ones compacted in ascending order.  Also clears the per-bhm counter
-// of the query-tile pass.
-__global__ void __launch_bounds__(256) meta_cols_kernel(const MetaParams p) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= p.BHm * p.T_k) return;
-  const int bhm = warp / p.T_k, kt = warp % p.T_k;
-  if (kt == 0 && lane == 0) p.done[bhm] = 0;
+// One list (a query tile's row over the key tiles, or a key tile's column over the query tiles)
+// built by a quad of four warps: warp w of the quad classifies positions [w c, (w + 1) c) with
+// c = 32 ceil(L / 128), 32 at a time, keeping the ballots of "non-skip" and "partial" in shared
+// memory (masks: 2 x L / 32 words for the quad); after the quad's named barrier each warp knows how
+// many entries the warps before it keep and writes its own entries (index << 1 | partial) in
+// ascending order.  class_of(idx) gives the class; on_class(idx, c) sees every classified position.
+template <typename ClassOf, typename OnClass>
+__device__ __forceinline__ int quad_list(int L, int wq, int lane, int bar_id, uint32_t* masks, int* counts,
+                                         int32_t* ent, ClassOf class_of, OnClass on_class) {
+  const unsigned below = (1u << lane) - 1u;
+  const int chunk = 32 * ((L + 127) / 128);
+  const int p0 = wq * chunk, p1 = min(p0 + chunk, L);
+  int count = 0;
+  for (int k0 = p0, it = 0; k0 < p1; k0 += 32, ++it) {
+    const int idx = k0 + lane;
+    int c = 0;
+    if (idx < p1) {
+      c = class_of(idx);
+      on_class(idx, c);
+    }
+    const unsigned keep = __ballot_sync(0xffffffffu, c != 0), part = __ballot_sync(0xffffffffu, c == 1);
+    if (lane == 0) {
+      masks[2 * (p0 / 32 + it)] = keep;
+      masks[2 * (p0 / 32 + it) + 1] = part;
+    }
+    count += __popc(keep);
+  }
+  if (lane == 0) counts[wq] = count;
+  named_bar_sync(bar_id, 128);
+  int base = 0;
+  for (int w = 0; w < wq; ++w) base += counts[w];
+  for (int k0 = p0, it = 0; k0 < p1; k0 += 32, ++it) {
+    const unsigned keep = masks[2 * (p0 / 32 + it)], part = masks[2 * (p0 / 32 + it) + 1];
+    if ((keep >> lane) & 1u) ent[base + __popc(keep & below)] = ((k0 + lane) << 1) | ((part >> lane) & 1u);
+    base += __popc(keep);
+  }
+  return counts[0] + counts[1] + counts[2] + counts[3];  // (read before the next use of counts)
+}
+
+// The same list built by one warp alone, in one pass (a running count of kept positions), for
+// launches large enough to fill the GPU with one warp per list.
+template <typename ClassOf, typename OnClass>
+__device__ __forceinline__ int warp_list(int L, int lane, int32_t* ent, ClassOf class_of, OnClass on_class) {
+  const unsigned below = (1u << lane) - 1u;
+  int count = 0;
+  for (int k0 = 0; k0 < L; k0 += 32) {
+    const int idx = k0 + lane;
+    int c = 0;
+    if (idx < L) {
+      c = class_of(idx);
+      on_class(idx, c);
+    }
+    const unsigned keep = __ballot_sync(0xffffffffu, c != 0);
+    if (c != 0) ent[count + __popc(keep & below)] = (idx << 1) | (c == 1 ? 1 : 0);
+    count += __popc(keep);
+  }
+  return count;
+}
+
+// Key-tile pass: W warps (a quad, or one) per (bhm, key tile), 8 / W tiles per CTA.  Min and max of
+// the four vectors over the tile's 128 columns (each warp reads its share, one column per lane;
+// a quad combines in shared memory), written to minmax, then the tile's column list over all query
+// tiles.  Also clears the per-bhm counter of the query-tile pass.
+constexpr int kColsThreads = 256;
+constexpr int kMaskWords = 2 * kOrderListMax / 32;
+template <int W>  // warps per key tile: 4 (a quad) or 1
+__global__ void __launch_bounds__(kColsThreads) meta_cols_kernel(const MetaParams p) {
+  constexpr int kLists = kColsThreads / 32 / W;  // key tiles per CTA
+  __shared__ int4 red[kLists][W][2];
+  __shared__ uint32_t masks[W == 4 ? kLists : 1][W == 4 ? kMaskWords : 1];
+  __shared__ int counts[kLists][4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, quad = warp / W, wq = warp % W;
+  const int64_t tile = (int64_t)blockIdx.x * kLists + quad;  // (bhm, key tile)
+  const bool live = tile < (int64_t)p.BHm * p.T_k;
+  const int bhm = live ? (int)(tile / p.T_k) : 0, kt = live ? (int)(tile % p.T_k) : 0;
+  if (live && kt == 0 && threadIdx.x == quad * 32 * W) p.done[bhm] = 0;
   const int32_t dflt[4] = {p.n_q, p.n_q, 0, 0};
   int32_t mn[4], mx[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     mn[c] = INT_MAX;
     mx[c] = INT_MIN;
-  }
-  const int64_t base = (int64_t)bhm * p.n_k;
-  const int64_t j0 = (int64_t)kt * kTile;
-  if (p.vec16) {
-    const int64_t j = j0 + 4 * lane;  // n_k % 4 == 0: a group of 4 is either inside or past the end
-    if (j < p.n_k) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        int4 v = make_int4(dflt[c], dflt[c], dflt[c], dflt[c]);
-        if (p.vec[c]) v = __ldg(reinterpret_cast<const int4*>(p.vec[c] + base + j));
-        mn[c] = min(min(v.x, v.y), min(v.z, v.w));
-        mx[c] = max(max(v.x, v.y), max(v.z, v.w));
-      }
-    }
-  } else {
-    for (int t = lane; t < kTile; t += 32) {
-      const int64_t j = j0 + t;
-      if (j >= p.n_k) break;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int32_t v = vec_at(p.vec[c], base + j, dflt[c]);
+    for (int t = wq * 32 + lane; t < kTile; t += 32 * W) {  // columns of this warp's share
+      const int64_t j = (int64_t)kt * kTile + t;
+      if (live && j < p.n_k) {
+        const int32_t v = vec_at(p.vec[c], (int64_t)bhm * p.n_k + j, dflt[c]);
         mn[c] = min(mn[c], v);
         mx[c] = max(mx[c], v);
       }
     }
-  }
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       mn[c] = min(mn[c], __shfl_xor_sync(0xffffffffu, mn[c], off));
       mx[c] = max(mx[c], __shfl_xor_sync(0xffffffffu, mx[c], off));
     }
   }
-  if (lane < 8) {
-    const int c = lane >> 1;
-    int32_t val = (lane & 1) ? mx[0] : mn[0];
-    // select without dynamic register indexing
-    val = (c == 1) ? ((lane & 1) ? mx[1] : mn[1]) : val;
-    val = (c == 2) ? ((lane & 1) ? mx[2] : mn[2]) : val;
-    val = (c == 3) ? ((lane & 1) ? mx[3] : mn[3]) : val;
-    p.minmax[((int64_t)bhm * p.T_k + kt) * 8 + lane] = val;
+  if (lane == 0) {
+    red[quad][wq][0] = make_int4(mn[0], mx[0], mn[1], mx[1]);
+    red[quad][wq][1] = make_int4(mn[2], mx[2], mn[3], mx[3]);
   }
-  // column list of this key tile
-  const int4 lo = make_int4(mn[0], mx[0], mn[1], mx[1]), hi = make_int4(mn[2], mx[2], mn[3], mx[3]);
-  const unsigned below = (1u << lane) - 1u;
-  int32_t* ent = p.col_entries + ((int64_t)bhm * p.T_k + kt) * p.T_q;
-  int count = 0;
-  for (int q0 = 0; q0 < p.T_q; q0 += 32) {
-    const int qt = q0 + lane;
-    int c = 0;
-    if (qt < p.T_q) {
-      const int64_t r0 = (int64_t)qt * kTile, r1 = (r0 + kTile < p.n_q) ? r0 + kTile : (int64_t)p.n_q;
-      c = classify(lo, hi, r0, r1);
-    }
-    const unsigned keep = __ballot_sync(0xffffffffu, c != 0);
-    if (c != 0) ent[count + __popc(keep & below)] = (qt << 1) | (c == 1 ? 1 : 0);
-    count += __popc(keep);
+  __syncthreads();
+  int4 lo = red[quad][0][0], hi = red[quad][0][1];
+#pragma unroll
+  for (int w = 1; w < W; ++w) {
+    const int4 a = red[quad][w][0], b = red[quad][w][1];
+    lo = make_int4(min(lo.x, a.x), max(lo.y, a.y), min(lo.z, a.z), max(lo.w, a.w));
+    hi = make_int4(min(hi.x, b.x), max(hi.y, b.y), min(hi.z, b.z), max(hi.w, b.w));
   }
-  if (lane == 0) p.col_count[(int64_t)bhm * p.T_k + kt] = count;
+  if (!live) return;  // (a whole quad: the barrier below is per quad)
+  if (wq == 0 && lane < 8) {
+    const int32_t v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    int32_t val = v[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) val = (lane == k) ? v[k] : val;  // select without dynamic indexing
+    p.minmax[tile * 8 + lane] = val;
+  }
+  int32_t* ent = p.col_entries + tile * p.T_q;
+  auto class_of = [&](int qt) { return classify(lo, hi, qt * kTile, tile_r1(qt * kTile, p.n_q)); };
+  auto none = [](int, int) {};
+  int n;
+  if constexpr (W == 4)
+    n = quad_list(p.T_q, wq, lane, 1 + quad, masks[quad], counts[quad], ent, class_of, none);
+  else
+    n = warp_list(p.T_q, lane, ent, class_of, none);
+  if (wq == 0 && lane == 0) p.col_count[tile] = n;
 }
 
 // Dispatch orders (longest first) of one (b, hm), by the CTA that finishes the query-tile pass
@@ -165,17 +216,21 @@ __device__ void sort_order(uint32_t* key, const int32_t* cost_a, bool pairs, int
   for (int i = tid; i < n; i += kT) out[i] = (int32_t)(0xFFFFu - (key[i] & 0xFFFFu));
 }
 
-// Query-tile pass: grid (ceil(T_q / 32), BHm), 1024 threads, one warp per query tile: its row of the
-// class matrix and its row list (key tiles scanned 32 at a time against the key-tile pass's min/max).
-// The CTA that completes a (b, hm) last also writes that (b, hm)'s two dispatch orders.
+// Query-tile pass: grid (ceil(T_q / (32 / W)), BHm), 1024 threads, W warps per query tile:
+// its row of the class matrix and its row list (quad_list over the key tiles, against the key-tile
+// pass's min/max staged in shared memory).  The CTA that completes a (b, hm) last also writes that
+// (b, hm)'s two dispatch orders.
+template <int W>  // warps per query tile: 4 (a quad) or 1
 __global__ void __launch_bounds__(kRowsThreads) meta_rows_kernel(const MetaParams p) {
+  constexpr int kLists = kRowsThreads / 32 / W;  // query tiles per CTA
   extern __shared__ int4 mm_smem[];  // this (b, hm)'s min/max, 2 x int4 per key tile (when it fits)
   __shared__ uint32_t key_f[kOrderMax / 2];
   __shared__ uint32_t key_b[kOrderMax];
+  __shared__ uint32_t masks[W == 4 ? kLists : 1][W == 4 ? kMaskWords : 1];
+  __shared__ int counts[kLists][4];
   __shared__ int last;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bhm = blockIdx.y, qt = blockIdx.x * (kRowsThreads / 32) + warp;
-  const unsigned below = (1u << lane) - 1u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, quad = warp / W, wq = warp % W;
+  const int bhm = blockIdx.y, qt = blockIdx.x * kLists + quad;
   const int4* mm_g = reinterpret_cast<const int4*>(p.minmax + (int64_t)bhm * p.T_k * 8);
   const bool staged = p.T_k <= kOrderMax;  // the launch gives 32 B of shared memory per key tile up to 4096
   if (staged) {
@@ -183,23 +238,18 @@ __global__ void __launch_bounds__(kRowsThreads) meta_rows_kernel(const MetaParam
     __syncthreads();
   }
   if (qt < p.T_q) {
-    const int64_t r0 = (int64_t)qt * kTile, r1 = (r0 + kTile < p.n_q) ? r0 + kTile : (int64_t)p.n_q;
+    const int r0 = qt * kTile, r1 = tile_r1(r0, p.n_q);
     const int4* mm = staged ? mm_smem : mm_g;
     uint8_t* cls = p.cls + ((int64_t)bhm * p.T_q + qt) * p.T_k;
     int32_t* ent = p.row_entries + ((int64_t)bhm * p.T_q + qt) * p.T_k;
-    int count = 0;
-    for (int k0 = 0; k0 < p.T_k; k0 += 32) {
-      const int kt = k0 + lane;
-      int c = 0;
-      if (kt < p.T_k) {
-        c = classify(mm[2 * kt], mm[2 * kt + 1], r0, r1);
-        cls[kt] = (uint8_t)c;
-      }
-      const unsigned keep = __ballot_sync(0xffffffffu, c != 0);
-      if (c != 0) ent[count + __popc(keep & below)] = (kt << 1) | (c == 1 ? 1 : 0);
-      count += __popc(keep);
-    }
-    if (lane == 0) p.row_count[(int64_t)bhm * p.T_q + qt] = count;
+    auto class_of = [&](int kt) { return classify(mm[2 * kt], mm[2 * kt + 1], r0, r1); };
+    auto store_class = [&](int kt, int c) { cls[kt] = (uint8_t)c; };
+    int n;
+    if constexpr (W == 4)
+      n = quad_list(p.T_k, wq, lane, 1 + quad, masks[quad], counts[quad], ent, class_of, store_class);
+    else
+      n = warp_list(p.T_k, lane, ent, class_of, store_class);
+    if (wq == 0 && lane == 0) p.row_count[(int64_t)bhm * p.T_q + qt] = n;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -331,17 +381,25 @@ fm_status fm_build_mask_meta(const fm_mask_desc* d, const int32_t* lts, const in
   p.n_k = d->n_k;
   p.T_q = (d->n_q + fm::kTile - 1) / fm::kTile;
   p.T_k = (d->n_k + fm::kTile - 1) / fm::kTile;
-  uintptr_t al = (uintptr_t)(d->n_k % 4);
-  for (int c = 0; c < 4; ++c) al |= reinterpret_cast<uintptr_t>(p.vec[c]) & 15u;
-  p.vec16 = al == 0;
   if (p.BHm > 65535) return FM_ERR_UNSUPPORTED;  // grid.y of the query-tile pass
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t warps_k = (int64_t)p.BHm * p.T_k;
-  fm::meta_cols_kernel<<<(unsigned)((warps_k + 7) / 8), 256, 0, s>>>(p);
+  // Lists per launch against the warps the GPU holds (148 SMs x 64): a quad of warps per list when
+  // one warp per list would leave most of the GPU idle, one warp per list otherwise.
+  constexpr int64_t kWarpsResident = 148 * 64;
+  const int64_t tiles_k = (int64_t)p.BHm * p.T_k, tiles_q = (int64_t)p.BHm * p.T_q;
+  if (4 * tiles_k <= 2 * kWarpsResident)
+    fm::meta_cols_kernel<4><<<(unsigned)((tiles_k + 1) / 2), fm::kColsThreads, 0, s>>>(p);
+  else
+    fm::meta_cols_kernel<1><<<(unsigned)((tiles_k + 7) / 8), fm::kColsThreads, 0, s>>>(p);
   // the query-tile pass stages the (b, hm)'s min/max in shared memory (32 B per key tile, <= 128 KiB)
   const int rows_smem = p.T_k <= fm::kOrderMax ? p.T_k * 32 : 0;
-  if (!fm::smem_opt_in<fm::meta_rows_kernel>(fm::kOrderMax * 32)) return FM_ERR_CUDA;  // + 24 KiB static
-  fm::meta_rows_kernel<<<dim3((unsigned)((p.T_q + 31) / 32), (unsigned)p.BHm), fm::kRowsThreads, rows_smem, s>>>(p);
+  if (4 * tiles_q <= 2 * kWarpsResident) {
+    if (!fm::smem_opt_in<fm::meta_rows_kernel<4>>(fm::kOrderMax * 32)) return FM_ERR_CUDA;  // + 33 KiB static
+    fm::meta_rows_kernel<4><<<dim3((unsigned)((p.T_q + 7) / 8), (unsigned)p.BHm), fm::kRowsThreads, rows_smem, s>>>(p);
+  } else {
+    if (!fm::smem_opt_in<fm::meta_rows_kernel<1>>(fm::kOrderMax * 32)) return FM_ERR_CUDA;
+    fm::meta_rows_kernel<1><<<dim3((unsigned)((p.T_q + 31) / 32), (unsigned)p.BHm), fm::kRowsThreads, rows_smem, s>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? FM_OK : FM_ERR_CUDA;
 }
 

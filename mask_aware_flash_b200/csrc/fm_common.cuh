@@ -439,6 +439,16 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// acc + (both bf16 halves of w), fp32 accumulate (mixed-precision adds)
+__device__ __forceinline__ float add_bf16x2_to_f32(uint32_t w, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 %0, lo, %2;\n\t"
+      "add.rn.f32.bf16 %0, hi, %0;\n\t}"
+      : "=f"(r) : "r"(w), "f"(acc));
+  return r;
+}
 
 // 2^x for a pair of fp32 values on the FMA / integer pipes (the MUFU unit's ex2
 // is the co-bottleneck of the forward softmax).  Argument reduction: n = round(x)

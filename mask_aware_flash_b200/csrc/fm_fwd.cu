@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + t * 256 + lane_addr, tO = tS + 128;
     const uint32_t has = (p.vec[0] ? 1u : 0u) | (p.vec[1] ? 2u : 0u) | (p.vec[2] ? 4u : 0u) | (p.vec[3] ? 8u : 0u);
-    float m_run = kNegInf, l_run = 0.f;
+    float m_run = kNegInf, l_run = 0.f, lq_run = 0.f;
     int j = 0, mcount = 0;
     bool ok = true;
     MergedList it{list0, list1, n0, n1, 0, 0, ragged_kt};
@@ -446,10 +446,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // P = 2^(s*scale - m) on pairs (f32x2), in two halves of 64 scores: each half is
         // stored (bf16 pairs over the first S columns) and published on its own barrier so
         // the PV product starts on the first half while the second is computed.
-        // rs: fp32 row sum of the unrounded P; it gives the LSE and normalises O (the bf16 P the PV
-        // product reads differs from it by one rounding per term, far inside the output's bf16 step).
+        // rs: exact fp32 row sum (LSE); rq: sum of the bf16-rounded P the PV product uses
+        // (O is normalised by it, so O stays a convex combination of V rows).
         const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-m_use, -m_use);
         uint64_t rs2[4] = {0, 0, 0, 0};
+        float rq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           // bf16: 32 packed pairs per half; fp32: 64 tf32-rounded values per half
@@ -470,10 +471,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const int k = (c >> 1) & 3;
             rs2[k] = add2(rs2[k], f2pack(p0, p1));
             if constexpr (F32) {
-              pk[c] = round_tf32(p0);
-              pk[c + 1] = round_tf32(p1);
+              const uint32_t w0 = round_tf32(p0), w1 = round_tf32(p1);
+              rq[k] += __uint_as_float(w0) + __uint_as_float(w1);
+              pk[c] = w0;
+              pk[c + 1] = w1;
             } else {
-              pk[c >> 1] = pack_bf16(p0, p1);
+              const uint32_t w = pack_bf16(p0, p1);
+              rq[k] = add_bf16x2_to_f32(w, rq[k]);
+              pk[c >> 1] = w;
             }
           }
           if (hh == 0 && __any_sync(0xffffffffu, move && j > 0)) {
@@ -501,7 +506,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!ok) break;
         const uint64_t rs2a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
         const float rs = f2lo(rs2a) + f2hi(rs2a);
+        const float rqs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
         l_run = l_run * alpha + rs;
+        lq_run = lq_run * alpha + rqs;
         m_run = m_new;
         ++j;
       } else if (has_mask) {
@@ -524,7 +531,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!have_o) record_failure(p.status, abort_flag, 6);
         tc_fence_after();
       }
-      const float inv = live ? 1.f / l_run : 0.f;
+      const float inv = live ? 1.f / lq_run : 0.f;
       // O tile staged in this tile's Q buffer (every S_t product has finished once O_DONE_t has
       // fired; the PV product does not read Q), 128-byte swizzle, then TMA-stored by one thread
       uint8_t* stage = smem + S::kQ + t * S::kTileBytes;
@@ -802,7 +809,7 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
     const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
     const uint32_t has = (p.vec[0] ? 1u : 0u) | (p.vec[1] ? 2u : 0u) | (p.vec[2] ? 4u : 0u) | (p.vec[3] ? 8u : 0u);
     const uint32_t tO = tmem + 256 + lane_addr;
-    float m_run = kNegInf, l_run = 0.f;
+    float m_run = kNegInf, l_run = 0.f, lq_run = 0.f;
     int mcount = 0;
     bool ok = true;
     int e = 0;
@@ -863,6 +870,7 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
       const float m_use = (m_new == kNegInf) ? 0.f : m_new;
       const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-m_use, -m_use);
       uint64_t rs2[4] = {0, 0, 0, 0};
+      float rq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[32];
@@ -881,7 +889,9 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
           }
           const int k = (c >> 1) & 3;
           rs2[k] = add2(rs2[k], f2pack(p0, p1));
-          pk[c >> 1] = pack_bf16(p0, p1);
+          const uint32_t w = pack_bf16(p0, p1);
+          rq[k] = add_bf16x2_to_f32(w, rq[k]);
+          pk[c >> 1] = w;
         }
         if (hh == 0 && __any_sync(0xffffffffu, move && e > 0)) {
           // O holds the sum over earlier tiles: wait for the last PV, rescale O in TMEM
@@ -904,6 +914,7 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
       if (!ok) break;
       const uint64_t rs2a = add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3]));
       l_run = l_run * alpha + (f2lo(rs2a) + f2hi(rs2a));
+      lq_run = lq_run * alpha + ((rq[0] + rq[1]) + (rq[2] + rq[3]));
       m_run = m_new;
     }
     if (!ok) record_failure(p.status, abort_flag, 24);
@@ -916,7 +927,7 @@ __global__ void __launch_bounds__(kFwd256Threads, 1)
       if (!have_o) record_failure(p.status, abort_flag, 25);
       tc_fence_after();
     }
-    const float inv = live ? 1.f / l_run : 0.f;
+    const float inv = live ? 1.f / lq_run : 0.f;
     uint8_t* stage = smem + S::kQ;
 #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {

@@ -81,11 +81,14 @@ def _check_meta(fm, vt, n_q, n_k):
             ce = meta.col_entries[b, hm].cpu().numpy()
             for kt in range(len(cc)):
                 np.testing.assert_array_equal(ce[kt, :cc[kt]], ref["col_entries"][kt, :cc[kt]])
-            # dispatch orders: longest first, ties by ascending index (stable sort on -cost)
+            # dispatch orders: longest first, ties by ascending index (stable sort on -cost); past
+            # 4096 tiles either way (sizes the attention kernels do not take) the identity order
             rcp = np.concatenate([ref["row_count"], [0]])[: 2 * ((len(rc) + 1) // 2)].reshape(-1, 2).sum(1)
-            np.testing.assert_array_equal(meta.fwd_order[b, hm].cpu().numpy(), np.argsort(-rcp, kind="stable"))
+            big = len(rc) > 4096 or len(cc) > 4096
+            np.testing.assert_array_equal(meta.fwd_order[b, hm].cpu().numpy(),
+                                          np.arange(len(rcp)) if big else np.argsort(-rcp, kind="stable"))
             np.testing.assert_array_equal(meta.bwd_order[b, hm].cpu().numpy(),
-                                          np.argsort(-ref["col_count"], kind="stable"))
+                                          np.arange(len(cc)) if big else np.argsort(-ref["col_count"], kind="stable"))
     return meta
 
 
@@ -105,6 +108,40 @@ def test_meta_bitexact_random_ragged(fm):
         _check_meta(fm, vt, n_q, n_k)
 
 
+def test_meta_bitexact_batched(fm):
+    # more than 148 x 32 query-tile lists in one launch: the query-tile pass takes four lists per warp
+    # (bit masks from each key tile's skip / partial ranges) instead of four warps per list
+    r = np.random.default_rng(11)
+    B, Hm, n_q, n_k = 2, 24, 16300, 13000
+    fams = list(synth.SWEEP_FAMILIES)
+    vecs = [np.empty((B, Hm, n_k), np.int32) for _ in range(4)]
+    for b in range(B):
+        for hm in range(Hm):
+            if (b * Hm + hm) % 3 == 2:  # random bounds, out-of-range values and int32 extremes included
+                for c in range(4):
+                    vecs[c][b, hm] = r.integers(-300, n_q + 300, n_k).astype(np.int32)
+                vecs[0][b, hm, :6] = [-2**31, 2**31 - 1, 0, n_q, n_q - 1, 128]
+                vecs[3][b, hm, 6:12] = [2**31 - 1, -2**31, n_q + 1, 127, 129, -1]
+            else:  # a sweep family laid out over n_k keys, rows clipped to n_q
+                spec = synth.make_family(fams[(b * Hm + hm) % len(fams)], n_k, 900 + b * Hm + hm)
+                for c, v in enumerate(spec.vectors()):
+                    vecs[c][b, hm] = v
+    assert B * Hm * ((n_q + 127) // 128) > 148 * 32
+    _check_meta(fm, [torch.from_numpy(v).cuda() for v in vecs], n_q, n_k)
+
+
+@pytest.mark.parametrize("n_q", [1000, 606300])
+def test_meta_unstaged_key_tiles(fm, n_q):
+    # more than 4096 key tiles: the query-tile pass reads the min/max from global memory instead of a
+    # shared-memory copy (n_q = 1000: four warps per list; 606300: 4737 query tiles, four lists per warp)
+    r = np.random.default_rng(12)
+    n_k = 530000
+    vecs = [r.integers(-100, n_q + 100, (1, 1, n_k)).astype(np.int32) for _ in range(4)]
+    vecs[1][0, 0, : n_k // 2] = n_q  # half the keys: lower interval to the end, so skip tiles exist
+    vecs[0][0, 0, : n_k // 2] = r.integers(0, n_q, n_k // 2)
+    _check_meta(fm, [torch.from_numpy(v).cuda() for v in vecs], n_q, n_k)
+
+
 def test_meta_null_vectors(fm):
     n = 512
     spec = synth.mask_causal(n)
@@ -113,16 +150,20 @@ def test_meta_null_vectors(fm):
     assert int(meta.tile_class.eq(1).sum()) == 4
 
 
-def test_meta_causal_128k_closed_form(fm):
+@pytest.mark.parametrize("Hm", [1, 8])
+def test_meta_causal_128k_closed_form(fm, Hm):
+    # Hm = 8: 8192 query-tile lists, the four-lists-per-warp form of the query-tile pass
     n = 131072
     T = n // 128
     spec = synth.mask_causal(n)
-    meta = fm.fm_build_mask_meta(*_vec_tensors(spec.vectors(), 1, 1, n), n_q=n)
-    cls = meta.tile_class[0, 0]
-    assert int(cls.eq(0).sum()) == T * (T - 1) // 2
-    assert int(cls.eq(1).sum()) == T
-    assert int(cls.eq(2).sum()) == T * (T - 1) // 2
-    assert int(meta.row_count.sum()) == T * (T + 1) // 2
+    meta = fm.fm_build_mask_meta(*_vec_tensors(spec.vectors(), 1, Hm, n), n_q=n)
+    for hm in range(Hm):
+        cls = meta.tile_class[0, hm]
+        assert int(cls.eq(0).sum()) == T * (T - 1) // 2
+        assert int(cls.eq(1).sum()) == T
+        assert int(cls.eq(2).sum()) == T * (T - 1) // 2
+        assert int(meta.row_count[0, hm].sum()) == T * (T + 1) // 2
+        assert int(meta.col_count[0, hm].sum()) == T * (T + 1) // 2
 
 
 # ---------------------------------------------------------------------------- localization

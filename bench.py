@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the phases eagerly instead of graph replays")
     ap.add_argument("--no-aux", action="store_true", help="skip the batched integer-pass measurement")
+    ap.add_argument("--aux-only", action="store_true",
+                    help="run only the batched integer-pass measurement (N=262144 localization and KV-chunk "
+                         "pairs, 16-head metadata) and print its JSON; not a bench line (profiling runs)")
     return ap.parse_args()
 
 
@@ -696,6 +699,17 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)))
+        return
+    if args.aux_only:
+        import torch
+        import mask_aware_flash_b200 as fm
+        from mask_aware_flash_b200 import _build
+        _build.build()
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        if rank == 0:
+            print(json.dumps({"integer_passes_batched": aux_localize(fm, torch, dev, torch.cuda.current_stream(),
+                                                                      peaks()[2])}))
         return
     if world > 1:
         import datetime

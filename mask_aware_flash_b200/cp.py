@@ -148,8 +148,12 @@ def cp_attention_forward(q, k, v, vecs, plan: ChunkPlan, scale: float, group=Non
         raise ValueError("the plan's rank count differs from the group's")
     L, n_ch = plan.chunk_len, plan.n_chunks
     n_loc = L * len(plan.owned[rank])
-    if q.shape[1] != n_loc or k.shape[1] != n_loc:
-        raise ValueError("q / k / v must hold this rank's rows")
+    if q.dim() != 4 or k.shape != v.shape or q.shape[1] != n_loc or k.shape[1] != n_loc or q.shape[0] != k.shape[0]:
+        raise ValueError("q [B, n_loc, H, D] and k, v [B, n_loc, H_kv, D] must hold this rank's rows")
+    if len(vecs) != 4 or any(x.dim() != 3 or x.shape[0] != q.shape[0] or x.shape[2] != plan.N for x in vecs):
+        raise ValueError("vecs must be the four global vectors [B, Hm, N] of the plan's sequence")
+    if any(x.device != q.device for x in (k, v, *vecs)):
+        raise ValueError("all tensors must be on the same device")
     B, _, H_kv, D = k.shape
     dev = q.device
     starts, lens = plan.starts_lens(rank)

@@ -70,8 +70,13 @@ class OracleOps:
 
 
 def _problem(N, B, H, D, mask, seed):
-    spec = synth.make_family(mask, N, seed)
-    vecs = [np.broadcast_to(x, (B, 1, N)).copy() for x in spec.vectors()]
+    if mask == "middle_rows_dead":  # rows [N/4, 3N/4) masked for every key: rank 1 of a 2-rank dual plan
+        lts, lte = np.full(N, N // 4, np.int32), np.full(N, 3 * N // 4, np.int32)
+        uts, ute = np.zeros(N, np.int32), np.arange(N, dtype=np.int32)  # causal elsewhere
+        raw = [lts, lte, uts, ute]
+    else:
+        raw = synth.make_family(mask, N, seed).vectors()
+    vecs = [np.broadcast_to(x, (B, 1, N)).copy() for x in raw]
     q, k, v, do = (synth.bf16_bits_to_f32(synth.normal_bf16_bits(seed, t, (B, N, H, D))) for t in (1, 2, 3, 4))
     return vecs, q, k, v, do
 
@@ -103,7 +108,8 @@ def _rank_main(rank, world, port, out_dir, N, mask, seed):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,mask", [(2, "causal_document"), (3, "sliding_window_2k"), (2, "full")])
+@pytest.mark.parametrize("world,mask", [(2, "causal_document"), (3, "sliding_window_2k"), (2, "full"),
+                                        (2, "middle_rows_dead")])
 def test_cp_exchange_matches_global_oracle(tmp_path, world, mask):
     N, seed = 768, 31
     port = _free_port()
@@ -130,10 +136,13 @@ def test_cp_exchange_matches_global_oracle(tmp_path, world, mask):
         loc = [oracle.localize(x[0, 0], *plan.starts_lens(r)) for x in vecs]
         pairs = oracle.kv_chunk_pairs(plan.chunk_len * 2, N, plan.chunk_len, *loc)
         np.testing.assert_array_equal(need[r], (pairs > 0).astype(np.uint8))
-    if mask != "full":
-        assert need.sum() < need.size  # chunks left out of the exchange
-    else:
+    if mask == "full":
         assert need.sum() == need.size
+    else:
+        assert need.sum() < need.size  # chunks left out of the exchange
+    if mask == "middle_rows_dead":  # rank 1 gathers nothing: its rows are O = 0, LSE = -inf, dQ = 0
+        assert need[1].sum() == 0 and res[1]["chunks"] == []
+        assert np.all(res[1]["o"] == 0) and np.all(np.isneginf(res[1]["lse"])) and np.all(res[1]["dq"] == 0)
 
 
 def test_chunk_plan_checks():
@@ -145,6 +154,38 @@ def test_chunk_plan_checks():
         cp.ChunkPlan(1024, 128, [[0, 1], [2, 3]])  # chunks 4..7 unowned
     with pytest.raises(ValueError):
         cp.ChunkPlan(1000, 125, [[0, 1, 2, 3], [4, 5, 6, 7]])  # chunk length not a multiple of 4
+
+
+def _rank_bad_args(rank, world, port, out_dir):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        plan = cp.ChunkPlan.dual(256, world)
+        q = torch.zeros(1, 128, 2, 16, dtype=torch.float64)
+        vt = [torch.zeros(1, 1, 256, dtype=torch.int32) for _ in range(4)]
+        errs = []
+        for args in ((q, q[:, :64], q, vt), (q, q, q, [x[..., :128] for x in vt]), (q, q, q, vt[:3])):
+            try:
+                cp.cp_attention_forward(*args, plan=plan, scale=0.25, ops=OracleOps())
+                errs.append("accepted")
+            except ValueError:
+                errs.append("rejected")
+        with pytest.raises(ValueError):  # a plan for another number of ranks
+            cp.cp_attention_forward(q, q, q, vt, cp.ChunkPlan.dual(256, world + 1), 0.25, ops=OracleOps())
+        with open(os.path.join(out_dir, f"e{rank}.txt"), "w") as f:
+            f.write(",".join(errs))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_cp_rejects_bad_arguments(tmp_path):
+    # every check fires on the host before any collective, on every rank
+    world = 2
+    mp.start_processes(_rank_bad_args, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn",
+                       join=True)
+    for r in range(world):
+        assert open(tmp_path / f"e{r}.txt").read() == "rejected,rejected,rejected"
 
 
 @pytest.mark.gpu

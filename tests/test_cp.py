@@ -44,7 +44,9 @@ class OracleOps:
 
     def _run(self, q, k, v, vecs, scale, do=None):
         B, n_q, H, D = q.shape
-        n_k = k.shape[1]
+        n_k, H_kv = k.shape[1], k.shape[2]
+        g = H // H_kv  # query heads per K/V head
+        k, v = k.repeat_interleave(g, dim=2), v.repeat_interleave(g, dim=2)
         Hm = vecs[0].shape[1]
         vv = [x.numpy() for x in vecs]
         o = np.zeros((B, n_q, H, D))
@@ -58,6 +60,8 @@ class OracleOps:
                 o[b, :, h], lse[b, h] = r["o"], r["lse"]
                 if do is not None:
                     dq[b, :, h], dk[b, :, h], dv[b, :, h] = r["dq"], r["dk"], r["dv"]
+        if g > 1:  # the gradient of a shared K/V head is the sum over its query heads
+            dk, dv = dk.reshape(B, n_k, H_kv, g, D).sum(3), dv.reshape(B, n_k, H_kv, g, D).sum(3)
         return o, lse, dq, dk, dv
 
     def attn_fwd(self, q, k, v, vecs, scale):
@@ -79,6 +83,68 @@ def _problem(N, B, H, D, mask, seed):
     vecs = [np.broadcast_to(x, (B, 1, N)).copy() for x in raw]
     q, k, v, do = (synth.bf16_bits_to_f32(synth.normal_bf16_bits(seed, t, (B, N, H, D))) for t in (1, 2, 3, 4))
     return vecs, q, k, v, do
+
+
+def _problem_multi(N, seed):
+    """B = 2, H = 4 query heads over H_kv = 2 K/V heads, per-head masks (Hm = H): a different
+    family per (b, h), so the need matrix is the union over every (b, mask head)."""
+    B, H, H_kv, D = 2, 4, 2, 16
+    fams = ["causal_document", "sliding_window_2k", "share_question", "prefix_lm_document"]
+    vecs = [np.empty((B, H, N), np.int32) for _ in range(4)]
+    for b in range(B):
+        for h in range(H):
+            for c, x in enumerate(synth.make_family(fams[(b + h) % 4], N, seed + 10 * b + h).vectors()):
+                vecs[c][b, h] = x
+    q, do = (synth.bf16_bits_to_f32(synth.normal_bf16_bits(seed, t, (B, N, H, D))) for t in (1, 4))
+    k, v = (synth.bf16_bits_to_f32(synth.normal_bf16_bits(seed, t, (B, N, H_kv, D))) for t in (2, 3))
+    return vecs, q, k, v, do
+
+
+def _rank_multi(rank, world, port, out_dir, N, seed):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        vecs, q, k, v, do = _problem_multi(N, seed)
+        plan = cp.ChunkPlan.dual(N, world)
+        rows = plan.rows(rank).numpy()
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rows])).double()  # noqa: E731
+        o, lse, ctx = cp.cp_attention_forward(t(q), t(k), t(v), [torch.from_numpy(x) for x in vecs], plan, 0.25,
+                                              ops=OracleOps())
+        dq, dk, dv = cp.cp_attention_backward(t(do), ctx)
+        with open(os.path.join(out_dir, f"m{rank}.pkl"), "wb") as f:
+            pickle.dump({"rows": rows, "o": o.numpy(), "lse": lse.numpy(), "dq": dq.numpy(), "dk": dk.numpy(),
+                         "dv": dv.numpy(), "need": ctx.need.numpy()}, f)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_cp_batched_per_head_masks_grouped_query(tmp_path):
+    N, seed, world = 512, 57, 2
+    mp.start_processes(_rank_multi, args=(world, _free_port(), str(tmp_path), N, seed), nprocs=world,
+                       start_method="spawn", join=True)
+    vecs, q, k, v, do = _problem_multi(N, seed)
+    ref = OracleOps()._run(*(torch.from_numpy(x) for x in (q, k, v)), [torch.from_numpy(x) for x in vecs], 0.25,
+                           torch.from_numpy(do))
+    o_ref, lse_ref, dq_ref, dk_ref, dv_ref = ref
+    tol = 1e-12 * max(np.abs(dq_ref).max(), np.abs(dk_ref).max(), np.abs(dv_ref).max())
+    plan = cp.ChunkPlan.dual(N, world)
+    for r in range(world):
+        res = pickle.load(open(tmp_path / f"m{r}.pkl", "rb"))
+        rows = res["rows"]
+        np.testing.assert_allclose(res["o"], o_ref[:, rows], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(res["lse"], lse_ref[:, :, rows], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(res["dq"], dq_ref[:, rows], rtol=0, atol=tol)
+        np.testing.assert_allclose(res["dk"], dk_ref[:, rows], rtol=0, atol=tol)
+        np.testing.assert_allclose(res["dv"], dv_ref[:, rows], rtol=0, atol=tol)
+        # need: any (b, mask head) of this rank's rows with unmasked pairs in the chunk
+        any_pairs = np.zeros(plan.n_chunks, bool)
+        for b in range(2):
+            for hm in range(4):
+                loc = [oracle.localize(x[b, hm], *plan.starts_lens(r)) for x in vecs]
+                any_pairs |= oracle.kv_chunk_pairs(2 * plan.chunk_len, N, plan.chunk_len, *loc) > 0
+        np.testing.assert_array_equal(res["need"][r], any_pairs.astype(np.uint8))
 
 
 def _free_port():

@@ -108,11 +108,13 @@ def test_meta_bitexact_random_ragged(fm):
         _check_meta(fm, vt, n_q, n_k)
 
 
-def test_meta_bitexact_batched(fm):
+@pytest.mark.parametrize("n_k", [13000, 12800])
+def test_meta_bitexact_batched(fm, n_k):
     # more than 148 x 32 query-tile lists in one launch: the query-tile pass takes four lists per warp
-    # (bit masks from each key tile's skip / partial ranges) instead of four warps per list
+    # (bit masks from each key tile's skip / partial ranges) instead of four warps per list; with
+    # n_k = 12800 (100 key tiles, a multiple of 4) its class bytes go out as packed 4-byte stores
     r = np.random.default_rng(11)
-    B, Hm, n_q, n_k = 2, 24, 16300, 13000
+    B, Hm, n_q = 2, 24, 16300
     fams = list(synth.SWEEP_FAMILIES)
     vecs = [np.empty((B, Hm, n_k), np.int32) for _ in range(4)]
     for b in range(B):
